@@ -1,0 +1,154 @@
+/*
+ * mmf.h — C ABI of the B200 (sm_100a) FusedBitLinear library (libmmf.so).
+ *
+ * FusedBitLinear is the projection used for every i/f/g/o and gate/down projection of the
+ * HGRNBit (MatMul-free) language model.  Sources (page title, section):
+ *   [P1] "matmulfreellm 評価: 行列積を消した HGRNBit を Transformers 互換で読む",
+ *        section "HGRNBit という層構成を読む" — FusedBitLinear holds an RMSNorm(eps=1e-08)
+ *        inside the projection; gate_proj is 2048 -> 11264, down_proj 5632 -> 2048, SiLU.
+ *   [P3] "MatMul-Free LM: Ternary-Gewichte statt Matrixmultiplikation im Transformer",
+ *        section "HGRNBit: was in einem Block tatsächlich passiert" — bias=False; the norm is
+ *        fused with the ternary projection.
+ *   [P4] "MatMul-freie LLMs: Zentrale Konzepte erklärt", sections "MatMul durch ternäre
+ *        Operationen ersetzen" (absmean quantisation of W to {-1,0,1}; products become adds
+ *        and subtracts) and "Kernkomponenten: MLGRU und GLU" (figure items 4 and 5; the GLU
+ *        paragraph).
+ *
+ * What one forward call computes, for x [T x K], norm weight g [K], packed weight codes c
+ * [N x K] with scale beta:
+ *   r_t     = sqrt(mean_k x_tk^2 + eps)                      (mean of squares in double,
+ *                                                              rounded once to float)
+ *   xhat_tk = (x_tk * (1/r_t)) * g_k                          (float)
+ *   gamma_t = max(max_k |xhat_tk|, 1e-5)
+ *   q_tk    = clamp(round_half_even(xhat_tk * (127/gamma_t)), -128, 127)      (int8)
+ *   acc_tn  = sum_{c_nk=+1} q_tk - sum_{c_nk=-1} q_tk                         (int32, exact)
+ *   y_tn    = acc_tn * (gamma_t/127) * beta                   (float, stored as f16 or f32)
+ * and the GLU form (gate_proj, N2 = 2I outputs) writes
+ *   h_ti    = silu(y_ti) * y_t,I+i,  silu(z) = z / (1 + exp(-z)),  i < I       (f16 or f32)
+ *
+ * Weight quantisation (once per weight matrix):
+ *   beta    = max( float( double(exact sum_{n,k} |W_nk|) / (N*K) ), 1e-5 )
+ *   c_nk    = clamp(round_half_even(W_nk / beta), -1, 1)      (division in float)
+ *
+ * Packed weight layout ("Wp", N x K/4 bytes, row-major, the library's own format — the pages
+ * fix none): the 16 codes k = 16G + 4i + j (i, j in 0..3) of group G of a row live in the
+ * little-endian 32-bit word at bytes 4G..4G+3 of that row, at bits 8j+2i and 8j+2i+1, as
+ * e = c + 1 (0, 1 or 2; the value 3 never occurs).  Equivalently byte j of a word holds the
+ * codes of k = j, j+4, j+8, j+12 of its group at bit pairs 0, 2, 4, 6.
+ *
+ * Conventions for every entry point:
+ *   - Memory: every pointer except those marked "host" is device memory owned by the caller.
+ *     The library allocates nothing per call.  Scratch comes from the caller's workspace.
+ *   - Alignment: every device pointer must be 16-byte aligned; workspaces 256-byte aligned.
+ *   - Shapes: row-major, contiguous.  K % 128 == 0 with 128 <= K <= 8192; N % 128 == 0;
+ *     1 <= T <= 16777216.
+ *   - Streams: `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on that stream and never synchronise the host, except
+ *     mmf_get_device_status.
+ *   - Errors: argument checks run on the host before any launch and return a status without
+ *     touching the device.  A failed launch returns MMF_ERR_CUDA.  A device-side wait that
+ *     runs past its time limit latches MMF_ERR_TIMEOUT in a device status word that
+ *     mmf_get_device_status reads; the kernel then returns instead of hanging.
+ *   - Threads: calls on distinct streams may run concurrently from distinct host threads as
+ *     long as they use distinct workspaces.
+ */
+#ifndef MMF_H_
+#define MMF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MMF_OK = 0,
+  MMF_ERR_INVALID_ARG = 1,        /* null pointer, bad dtype, non-positive eps, ... */
+  MMF_ERR_UNSUPPORTED_SHAPE = 2,  /* a dimension outside the limits above */
+  MMF_ERR_ALIGNMENT = 3,          /* a pointer not aligned as required */
+  MMF_ERR_CUDA = 4,               /* a CUDA runtime or driver call failed */
+  MMF_ERR_TIMEOUT = 5,            /* a device-side wait ran past its limit */
+  MMF_ERR_WORKSPACE = 6           /* workspace missing or smaller than required */
+} mmf_status;
+
+typedef enum { MMF_F32 = 0, MMF_F16 = 1 } mmf_dtype;
+
+/* ---- weight quantisation ([P4] "MatMul durch ternäre Operationen ersetzen") ------------- */
+
+/* Workspace bytes mmf_quantize_weights needs for an N x K matrix (a fixed 4 KiB). */
+size_t mmf_quantize_weights_workspace_bytes(int64_t N, int64_t K);
+
+/* W [N x K] (wdt: f32 or f16, finite values) -> Wp [N x K/4] packed codes and beta (one
+ * float, device).  Runs three kernels: an exact sum of |W|, a one-thread finalisation of
+ * beta, and the encode+pack pass.  ws must hold mmf_quantize_weights_workspace_bytes. */
+mmf_status mmf_quantize_weights(const void* W, mmf_dtype wdt, int64_t N, int64_t K,
+                                uint8_t* Wp, float* beta, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/* Encode+pack pass alone, with beta given (device float): the codes of W under that beta.
+ * Lets callers (and the parity tests) fix beta and compare codes bit for bit. */
+mmf_status mmf_ternary_encode(const void* W, mmf_dtype wdt, int64_t N, int64_t K,
+                              const float* beta, uint8_t* Wp, void* stream);
+
+/* ---- forward ([P1], [P3]; [P4] figure items 4 and 5) ------------------------------------ */
+
+/* Workspace bytes one forward call with T tokens, K inputs and N outputs needs: the int8
+ * activation codes [T x K], gamma [T] and the code row sums [T], each 256-byte aligned. */
+size_t mmf_forward_workspace_bytes(int64_t T, int64_t K, int64_t N);
+
+/* y [T x N] = FusedBitLinear(x [T x K]).  xdt: f32 or f16.  norm_w: K floats or NULL
+ * (all ones).  eps > 0 (the model uses 1e-8).  Wp/beta from mmf_quantize_weights.
+ * ydt: f32 or f16.  Two launches on `stream`: RMSNorm + activation quantisation, then the
+ * tensor-core ternary contraction with the dequantisation epilogue. */
+mmf_status mmf_bitlinear_forward(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
+                                 const float* norm_w, float eps, const uint8_t* Wp,
+                                 const float* beta, int64_t N, void* y, mmf_dtype ydt,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* gate_proj with the fused SiLU-GLU epilogue ([P4] GLU paragraph; [P1] 2I -> I).
+ * Wp holds the whole 2I x K gate_proj (N2 = 2I rows, one beta); h [T x I] receives
+ * silu(first half) * second half.  N2 % 128 == 0. */
+mmf_status mmf_bitlinear_glu_forward(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
+                                     const float* norm_w, float eps, const uint8_t* Wp,
+                                     const float* beta, int64_t N2, void* h, mmf_dtype hdt,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---- the two halves of the forward, exported for bit-exact checks ------------------------ */
+
+/* RMSNorm + activation quantisation alone: A [T x K] int8, gamma [T], rowsum [T] (the plain
+ * sum of each row of A; may be NULL). */
+mmf_status mmf_quantize_activations(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
+                                    const float* norm_w, float eps, int8_t* A, float* gamma,
+                                    int32_t* rowsum, void* stream);
+
+/* acc [T x N] int32 = ternary accumulation of given codes A [T x K] against Wp.  Exact.
+ * ws must hold mmf_forward_workspace_bytes(T, K, N). */
+mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int64_t K, const uint8_t* Wp,
+                                      int64_t N, int32_t* acc, void* ws, size_t ws_bytes,
+                                      void* stream);
+
+/* ---- status ------------------------------------------------------------------------------ */
+
+/* Reads and clears the device status word of the current device (synchronises the device).
+ * Returns MMF_OK, MMF_ERR_TIMEOUT if a kernel gave up on a wait since the last read, or
+ * MMF_ERR_CUDA if the read itself failed. */
+mmf_status mmf_get_device_status(void);
+
+/* Launches one block whose single wait can never be satisfied and must give up after
+ * `limit_ns` nanoseconds (1e3 <= limit_ns <= 1e9); the next mmf_get_device_status then
+ * returns MMF_ERR_TIMEOUT.  Exercises the same bounded-wait routine the pipelined kernels
+ * use, without any copy or tensor-core work in flight. */
+mmf_status mmf_debug_wait_timeout_probe(uint64_t limit_ns, void* stream);
+
+/* Human-readable name of a status. */
+const char* mmf_status_string(mmf_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int mmf_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MMF_H_ */

@@ -1,0 +1,217 @@
+"""Python binding of libmmf.so, the B200 FusedBitLinear library.
+
+Argument marshalling only: every step of the projection runs in the library's CUDA kernels.
+PyTorch supplies device memory (``tensor.data_ptr()``) and streams
+(``torch.cuda.current_stream().cuda_stream``).  There is no CPU path: if the library or a GPU
+is missing, calls raise.
+
+The functions named ``mmf_*`` mirror the C ABI in ``include/mmf.h`` one to one and take
+tensors that the caller owns.  ``quantize_weights``, ``bitlinear_forward`` and
+``bitlinear_glu_forward`` are conveniences that allocate the outputs and the workspace with
+torch and then call the same entry points.
+"""
+import ctypes
+import os
+
+__all__ = [
+    "MMFError", "lib", "lib_path",
+    "mmf_quantize_weights_workspace_bytes", "mmf_quantize_weights", "mmf_ternary_encode",
+    "mmf_forward_workspace_bytes", "mmf_bitlinear_forward", "mmf_bitlinear_glu_forward",
+    "mmf_quantize_activations", "mmf_ternary_accumulate_i32", "mmf_get_device_status",
+    "mmf_debug_wait_timeout_probe", "mmf_status_string", "mmf_version",
+    "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
+    "MMF_F32", "MMF_F16", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libmmf.so")
+
+MMF_F32 = 0
+MMF_F16 = 1
+STATUS = {
+    0: "MMF_OK", 1: "MMF_ERR_INVALID_ARG", 2: "MMF_ERR_UNSUPPORTED_SHAPE",
+    3: "MMF_ERR_ALIGNMENT", 4: "MMF_ERR_CUDA", 5: "MMF_ERR_TIMEOUT", 6: "MMF_ERR_WORKSPACE",
+}
+
+
+class MMFError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libmmf.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise OSError(f"{lib_path} is missing: run ternary_weight_lm_b200/build.py")
+        L = ctypes.CDLL(lib_path)
+        P, I64, F, SZ, I = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
+                            ctypes.c_int)
+        sigs = {
+            "mmf_quantize_weights_workspace_bytes": ([I64, I64], SZ),
+            "mmf_quantize_weights": ([P, I, I64, I64, P, P, P, SZ, P], I),
+            "mmf_ternary_encode": ([P, I, I64, I64, P, P, P], I),
+            "mmf_forward_workspace_bytes": ([I64, I64, I64], SZ),
+            "mmf_bitlinear_forward": ([P, I, I64, I64, P, F, P, P, I64, P, I, P, SZ, P], I),
+            "mmf_bitlinear_glu_forward": ([P, I, I64, I64, P, F, P, P, I64, P, I, P, SZ, P], I),
+            "mmf_quantize_activations": ([P, I, I64, I64, P, F, P, P, P, P], I),
+            "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
+            "mmf_get_device_status": ([], I),
+            "mmf_debug_wait_timeout_probe": ([ctypes.c_uint64, P], I),
+            "mmf_status_string": ([I], ctypes.c_char_p),
+            "mmf_version": ([], I),
+        }
+        for name, (args, res) in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------------------ marshalling
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dt(t):
+    import torch
+    if t.dtype == torch.float32:
+        return MMF_F32
+    if t.dtype == torch.float16:
+        return MMF_F16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn, code):
+    if code != 0:
+        raise MMFError(fn, code)
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+# ------------------------------------------------------------------------------ C ABI mirror
+def mmf_quantize_weights_workspace_bytes(N, K):
+    return lib().mmf_quantize_weights_workspace_bytes(N, K)
+
+
+def mmf_quantize_weights(W, Wp, beta, ws, stream=None):
+    N, K = W.shape
+    _check("mmf_quantize_weights", lib().mmf_quantize_weights(
+        _ptr(W), _dt(W), N, K, _ptr(Wp), _ptr(beta), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def mmf_ternary_encode(W, beta, Wp, stream=None):
+    N, K = W.shape
+    _check("mmf_ternary_encode", lib().mmf_ternary_encode(
+        _ptr(W), _dt(W), N, K, _ptr(beta), _ptr(Wp), _stream(stream)))
+
+
+def mmf_forward_workspace_bytes(T, K, N):
+    return lib().mmf_forward_workspace_bytes(T, K, N)
+
+
+def mmf_bitlinear_forward(x, norm_w, eps, Wp, beta, N, y, ws, stream=None):
+    T, K = x.shape
+    _check("mmf_bitlinear_forward", lib().mmf_bitlinear_forward(
+        _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(Wp), _ptr(beta), N, _ptr(y),
+        _dt(y), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def mmf_bitlinear_glu_forward(x, norm_w, eps, Wp, beta, N2, h, ws, stream=None):
+    T, K = x.shape
+    _check("mmf_bitlinear_glu_forward", lib().mmf_bitlinear_glu_forward(
+        _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(Wp), _ptr(beta), N2, _ptr(h),
+        _dt(h), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def mmf_quantize_activations(x, norm_w, eps, A, gamma, rowsum=None, stream=None):
+    T, K = x.shape
+    _check("mmf_quantize_activations", lib().mmf_quantize_activations(
+        _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(A), _ptr(gamma), _ptr(rowsum),
+        _stream(stream)))
+
+
+def mmf_ternary_accumulate_i32(A, Wp, N, acc, ws, stream=None):
+    T, K = A.shape
+    _check("mmf_ternary_accumulate_i32", lib().mmf_ternary_accumulate_i32(
+        _ptr(A), T, K, _ptr(Wp), N, _ptr(acc), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def mmf_get_device_status():
+    """Status code (int) of the device status word; reading clears it."""
+    return lib().mmf_get_device_status()
+
+
+def mmf_debug_wait_timeout_probe(limit_ns, stream=None):
+    _check("mmf_debug_wait_timeout_probe",
+           lib().mmf_debug_wait_timeout_probe(int(limit_ns), _stream(stream)))
+
+
+def mmf_status_string(code):
+    return lib().mmf_status_string(code).decode()
+
+
+def mmf_version():
+    return lib().mmf_version()
+
+
+# ------------------------------------------------------------------------------ conveniences
+def workspace(nbytes, device="cuda"):
+    import torch
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def quantize_weights(W, stream=None):
+    """W [N,K] (fp32/fp16, CUDA) -> (Wp uint8 [N, K/4], beta float32 [1])."""
+    import torch
+    N, K = W.shape
+    Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    beta = torch.empty(1, dtype=torch.float32, device=W.device)
+    ws = workspace(mmf_quantize_weights_workspace_bytes(N, K), W.device)
+    mmf_quantize_weights(W, Wp, beta, ws, stream)
+    return Wp, beta
+
+
+def bitlinear_forward(x, Wp, beta, norm_w=None, eps=1e-8, out_dtype=None, ws=None,
+                      stream=None):
+    import torch
+    T, K = x.shape
+    N = Wp.shape[0]
+    y = torch.empty((T, N), dtype=out_dtype or x.dtype, device=x.device)
+    if ws is None:
+        ws = workspace(mmf_forward_workspace_bytes(T, K, N), x.device)
+    mmf_bitlinear_forward(x, norm_w, eps, Wp, beta, N, y, ws, stream)
+    return y
+
+
+def bitlinear_glu_forward(x, Wp, beta, norm_w=None, eps=1e-8, out_dtype=None, ws=None,
+                          stream=None):
+    import torch
+    T, K = x.shape
+    N2 = Wp.shape[0]
+    h = torch.empty((T, N2 // 2), dtype=out_dtype or x.dtype, device=x.device)
+    if ws is None:
+        ws = workspace(mmf_forward_workspace_bytes(T, K, N2), x.device)
+    mmf_bitlinear_glu_forward(x, norm_w, eps, Wp, beta, N2, h, ws, stream)
+    return h

@@ -1,0 +1,228 @@
+// RMSNorm inside the projection + per-token absmax int8 activation quantisation.
+//
+// "MatMul-freie LLMs: Zentrale Konzepte erklärt", section "Kernkomponenten: MLGRU und GLU",
+// figure item 5: RMSNorm normalises the activations before they are quantised; the
+// FusedBitLinear layers of the HGRNBit tree carry RMSNorm(eps=1e-08) inside the projection
+// ("matmulfreellm 評価 ...", section "HGRNBit という層構成を読む").
+//
+// One CTA of 128 threads per token row.  The row is read once from HBM with 16-byte loads and
+// kept in registers across the three block reductions it needs: sum of squares (double),
+// max |xhat| (float) and the sum of the int8 codes (int, used by the contraction to undo the
+// +1 offset of the packed weight codes).  Every rounding decision uses the same single-
+// precision operation sequence as the definition: ms = float(sum/K), r = sqrt(ms + eps),
+// inv = 1/r, xhat = (x * inv) * g, s = 127/gamma, q = round_half_even(xhat * s).
+#include <cuda_fp16.h>
+
+#include "kernels.cuh"
+
+namespace mmf {
+namespace {
+
+constexpr int kAqThreads = 128;
+constexpr int kAqWarps = kAqThreads / 32;
+
+template <typename TIn>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int E = 4;
+  __device__ static void load(const void* p, float (&v)[E]) {
+    float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+};
+template <>
+struct Vec<__half> {
+  static constexpr int E = 8;
+  __device__ static void load(const void* p, float (&v)[E]) {
+    uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const __half2* h = reinterpret_cast<const __half2*>(&a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __half22float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+};
+
+__device__ __forceinline__ double block_sum_d(double v, double* sh) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) sh[w] = v;
+  __syncthreads();
+  double t = 0.0;
+#pragma unroll
+  for (int i = 0; i < kAqWarps; ++i) t += sh[i];
+  __syncthreads();
+  return t;
+}
+
+__device__ __forceinline__ float block_max_f(float v, float* sh) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) sh[w] = v;
+  __syncthreads();
+  float t = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kAqWarps; ++i) t = fmaxf(t, sh[i]);
+  __syncthreads();
+  return t;
+}
+
+__device__ __forceinline__ int block_sum_i(int v, int* sh) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) sh[w] = v;
+  __syncthreads();
+  int t = 0;
+#pragma unroll
+  for (int i = 0; i < kAqWarps; ++i) t += sh[i];
+  __syncthreads();
+  return t;
+}
+
+__device__ __forceinline__ uint32_t code_byte(float xh, float s) {
+  int q = __float2int_rn(__fmul_rn(xh, s));
+  q = max(-128, min(127, q));
+  return static_cast<uint32_t>(q) & 0xFFu;
+}
+
+// MAXV = most 16-byte vectors one thread holds: K <= kAqThreads * MAXV * E.
+template <typename TIn, int MAXV>
+__global__ void __launch_bounds__(kAqThreads)
+act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, float eps,
+                 int8_t* __restrict__ A, float* __restrict__ gamma,
+                 int32_t* __restrict__ rowsum) {
+  using V = Vec<TIn>;
+  constexpr int E = V::E;
+  __shared__ double sh_d[kAqWarps];
+  __shared__ float sh_f[kAqWarps];
+  __shared__ int sh_i[kAqWarps];
+
+  const int64_t row = blockIdx.x;
+  const int nvec = K / E;
+  const TIn* xr = x + row * static_cast<int64_t>(K);
+
+  float v[MAXV][E];
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int vi = threadIdx.x + i * kAqThreads;
+    if (vi < nvec) {
+      V::load(xr + static_cast<int64_t>(vi) * E, v[i]);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const double d = static_cast<double>(v[i][e]);
+        ss = __fma_rn(d, d, ss);   // d*d is exact in double: same as an add of the square
+      }
+    }
+  }
+  ss = block_sum_d(ss, sh_d);
+  const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
+  const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int vi = threadIdx.x + i * kAqThreads;
+    if (vi < nvec) {
+      float gk[E];
+      if (g != nullptr) {
+#pragma unroll
+        for (int e = 0; e < E; e += 4) {
+          float4 t = __ldg(reinterpret_cast<const float4*>(g + vi * E + e));
+          gk[e] = t.x; gk[e + 1] = t.y; gk[e + 2] = t.z; gk[e + 3] = t.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) gk[e] = 1.0f;
+      }
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        v[i][e] = __fmul_rn(__fmul_rn(v[i][e], inv_r), gk[e]);
+        amax = fmaxf(amax, fabsf(v[i][e]));
+      }
+    }
+  }
+  amax = block_max_f(amax, sh_f);
+  const float gm = fmaxf(amax, 1e-5f);
+  const float s = __fdiv_rn(127.0f, gm);
+
+  int rs = 0;
+  int8_t* ar = A + row * static_cast<int64_t>(K);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int vi = threadIdx.x + i * kAqThreads;
+    if (vi < nvec) {
+      uint32_t w[E / 4];
+#pragma unroll
+      for (int c = 0; c < E / 4; ++c) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const uint32_t cb = code_byte(v[i][4 * c + b], s);
+          rs += static_cast<int>(static_cast<int8_t>(cb));
+          word |= cb << (8 * b);
+        }
+        w[c] = word;
+      }
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint2*>(ar + vi * E) = make_uint2(w[0], w[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(ar + vi * E) = w[0];
+      }
+    }
+  }
+  rs = block_sum_i(rs, sh_i);
+  if (threadIdx.x == 0) {
+    gamma[row] = gm;
+    if (rowsum != nullptr) rowsum[row] = rs;
+  }
+}
+
+__global__ void __launch_bounds__(kAqThreads)
+rowsum_kernel(const int8_t* __restrict__ A, int K, int32_t* __restrict__ rowsum) {
+  __shared__ int sh_i[kAqWarps];
+  const int64_t row = blockIdx.x;
+  const int8_t* ar = A + row * static_cast<int64_t>(K);
+  int s = 0;
+  for (int i = threadIdx.x * 16; i < K; i += kAqThreads * 16) {
+    int4 q = *reinterpret_cast<const int4*>(ar + i);
+    const int w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) s += static_cast<int8_t>((w[j] >> (8 * b)) & 0xFF);
+    }
+  }
+  s = block_sum_i(s, sh_i);
+  if (threadIdx.x == 0) rowsum[row] = s;
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const void* x, int xdt, int64_t T, int K, const float* g, float eps,
+                             int8_t* A, float* gamma, int32_t* rowsum, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(T));
+  if (xdt == kInF16) {
+    // 8 halves per vector: K <= 128 * 8 * 8 = 8192
+    act_quant_kernel<__half, 8><<<grid, kAqThreads, 0, s>>>(
+        reinterpret_cast<const __half*>(x), K, g, eps, A, gamma, rowsum);
+  } else {
+    // 4 floats per vector: K <= 128 * 16 * 4 = 8192
+    act_quant_kernel<float, 16><<<grid, kAqThreads, 0, s>>>(
+        reinterpret_cast<const float*>(x), K, g, eps, A, gamma, rowsum);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rowsum(const int8_t* A, int64_t T, int K, int32_t* rowsum, cudaStream_t s) {
+  rowsum_kernel<<<static_cast<unsigned>(T), kAqThreads, 0, s>>>(A, K, rowsum);
+  return cudaGetLastError();
+}
+
+}  // namespace mmf

@@ -1,0 +1,418 @@
+// Ternary contraction on the 5th-generation tensor cores (tcgen05, kind::i8) with the
+// dequantisation and SiLU-GLU epilogues.
+//
+// "MatMul-freie LLMs: Zentrale Konzepte erklärt": section "MatMul durch ternäre Operationen
+// ersetzen" (weights in {-1,0,1}: products become adds and subtracts) and figure item 4
+// (scaled ternary accumulation); the GLU paragraph (one branch through SiLU times the other).
+//
+// Orientation ("swap AB"): the MMA's M side is 128 weight rows and its N side is BN tokens,
+// so one kernel serves a single decode token (N = 16) up to prefill tiles (N = 256).
+//   A (u8, TMEM)  : unpacked weight codes e = c + 1 in {0,1,2}, one TMEM lane per weight row
+//   B (s8, SMEM)  : int8 activation codes, loaded by TMA with the 128-byte swizzle
+//   D (s32, TMEM) : sum_k e_nk q_tk; the epilogue subtracts sum_k q_tk (computed by the
+//                   activation pre-pass), giving exactly sum_k c_nk q_tk.
+// The packed weights reach shared memory by TMA at 2 bits per weight (32-byte swizzle); four
+// "unpack" warps, one thread per weight row, turn each 32-bit word of 16 codes into four
+// 32-bit words of int8 codes with one shift and one mask each (the packing puts code 4i + j
+// at bits 8j + 2i), and store them straight into TMEM with tcgen05.st.  Unpacked weights
+// never touch shared memory, so shared-memory traffic stays at the packed 2 bits per weight.
+//
+// Warp roles (192 threads): warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one
+// thread), warps 2-5 unpack and then run the epilogue (TMEM lane quarter = warp % 4).
+// Every mbarrier wait is bounded (mbar_wait_bounded): on a timeout the block records
+// kStatusTimeout, stops, drains the copies and MMAs it issued, frees TMEM and returns.
+#include <cuda_fp16.h>
+
+#include <mutex>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace mmf {
+namespace {
+
+constexpr int kKB = 128;                       // K elements per pipeline stage
+constexpr int kWRowBytes = kKB / 4;            // packed bytes of one weight row per stage
+constexpr int kWHalfBytes = 64 * kWRowBytes;   // one TMA box: 64 rows x 32 bytes
+constexpr int kWStageBytes = 2 * kWHalfBytes;  // 128 rows
+constexpr int kASlots = 4;                     // TMEM slots of unpacked weights (32 columns)
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr uint64_t kDrainNs = 2000000000ull;
+
+template <int BN>
+struct Cfg {
+  static constexpr int kActStage = BN * kKB;               // int8 activation tile
+  static constexpr int kStage = kActStage + kWStageBytes;
+  static constexpr int kStagesRaw = (200 * 1024) / kStage;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kTmemCols = BN <= 128 ? 256 : 512;
+  static constexpr int kACol0 = BN <= 128 ? 128 : 256;     // first TMEM column of A slots
+  static constexpr int kChunk = BN < 32 ? BN : 32;         // epilogue token columns per pass
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kASlots + 1);
+  // Request at least ~116 KB so only one CTA lives on an SM (its TMEM allocation never waits).
+  static constexpr int kSmemUsed = 1024 + kStages * kStage + kBarBytes;
+  static constexpr int kSmem = kSmemUsed < 118 * 1024 ? 118 * 1024 : kSmemUsed;
+  static_assert(kStages >= 2, "pipeline needs two stages");
+  static_assert(kChunk * 128 * 4 <= kStages * kActStage, "epilogue staging must fit");
+};
+
+struct Params {
+  int64_t T;
+  int K;
+  int rows;       // weight rows addressed by the tensor map
+  int glu;
+  int half;       // GLU: I (row offset of the multiplier half)
+  int out_mode;
+  int ldy;        // output row stride in elements
+  const float* gamma;
+  const int32_t* rowsum;
+  const float* beta;
+  void* y;
+  unsigned* status;
+  uint64_t wait_limit_ns;
+};
+
+// One 32-bit word of 16 packed codes -> four words of four int8 codes e = c + 1 in K order.
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t* out) {
+  out[0] = w & 0x03030303u;
+  out[1] = (w >> 2) & 0x03030303u;
+  out[2] = (w >> 4) & 0x03030303u;
+  out[3] = (w >> 6) & 0x03030303u;
+}
+
+__device__ __forceinline__ float sigmoid_mul(float g, float u) {
+  return __fdividef(g, 1.0f + expf(-g)) * u;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
+                    const Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* s_act = smem;
+  uint8_t* s_w = smem + C::kStages * C::kActStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + C::kStages * kWStageBytes);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkb = p.K / kKB;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * BN;
+  int r0, r1;  // first weight row of each 64-row half of the tile
+  if (p.glu) {
+    r0 = blockIdx.x * 64;
+    r1 = p.half + blockIdx.x * 64;
+  } else {
+    r0 = blockIdx.x * 128;
+    r1 = r0 + 64;
+  }
+
+  auto full = [&](int s) { return smem_u32(bars + s); };
+  auto empty = [&](int s) { return smem_u32(bars + C::kStages + s); };
+  auto afull = [&](int j) { return smem_u32(bars + 2 * C::kStages + j); };
+  auto aempty = [&](int j) { return smem_u32(bars + 2 * C::kStages + kASlots + j); };
+  const uint32_t accfull = smem_u32(bars + 2 * C::kStages + 2 * kASlots);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1 + 4);   // the MMA commit + the four unpack warps
+    }
+    for (int j = 0; j < kASlots; ++j) {
+      mbar_init(afull(j), 4);
+      mbar_init(aempty(j), 1);
+    }
+    mbar_init(accfull, 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_a);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();   // weights: each byte is used once
+      const uint64_t pol_a = l2_policy_evict_last();    // activations: reused by every tile
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % C::kStages;
+        if (kb >= C::kStages &&
+            !mbar_wait_bounded(empty(s), ((kb / C::kStages) - 1) & 1, p.wait_limit_ns,
+                               abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(full(s), C::kStage);
+        tma_load_2d(smem_u32(s_act + s * C::kActStage), &tm_a, full(s), kb * kKB,
+                    static_cast<int32_t>(t0), pol_a);
+        uint8_t* wdst = s_w + s * kWStageBytes;
+        tma_load_2d(smem_u32(wdst), &tm_w, full(s), kb * kWRowBytes, r0, pol_w);
+        tma_load_2d(smem_u32(wdst + kWHalfBytes), &tm_w, full(s), kb * kWRowBytes, r1, pol_w);
+        issued = kb + 1;
+      }
+      // Every copy this thread started must land before the block may exit.
+      for (int kb = issued > C::kStages ? issued - C::kStages : 0; kb < issued; ++kb)
+        mbar_wait_bounded(full(kb % C::kStages), (kb / C::kStages) & 1, kDrainNs, nullptr,
+                          p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % C::kStages, j = kb % kASlots;
+        if (!mbar_wait_bounded(full(s), (kb / C::kStages) & 1, p.wait_limit_ns, abort_flag,
+                               p.status))
+          break;
+        if (!mbar_wait_bounded(afull(j), (kb / kASlots) & 1, p.wait_limit_ns, abort_flag,
+                               p.status))
+          break;
+        tc_fence_after();
+        const uint32_t b0 = smem_u32(s_act + s * C::kActStage);
+#pragma unroll
+        for (int kk = 0; kk < kKB / 32; ++kk) {
+          tc_mma_i8_ts(tmem, tmem + C::kACol0 + j * 32 + kk * 8, smem_desc_kmajor_sw128(b0 + kk * 32),
+                       idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        tc_commit(empty(s));
+        tc_commit(aempty(j));
+      }
+      // Signals the epilogue; in the abort path it also tells this thread when the MMAs it
+      // issued have finished, so TMEM is not freed under them.
+      tc_commit(accfull);
+      mbar_wait_bounded(accfull, 0, kDrainNs, nullptr, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------------ unpack + epilogue
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;         // tile row = TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    // Wait outcomes are made warp-uniform (__all_sync) before the .sync.aligned tcgen05
+    // instructions, and the epilogue is entered by all four warps or by none.
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % C::kStages, j = kb % kASlots;
+      bool w = mbar_wait_bounded(full(s), (kb / C::kStages) & 1, p.wait_limit_ns, abort_flag,
+                                 p.status);
+      if (!__all_sync(0xFFFFFFFFu, w)) {
+        ok = false;
+        break;
+      }
+      // Row r of the 32-byte-swizzled tile: 16-byte chunk c sits at c ^ ((r >> 2) & 1).
+      const uint8_t* wrow = s_w + s * kWStageBytes + r * kWRowBytes;
+      const int sw = (r >> 2) & 1;
+      const uint4 lo = *reinterpret_cast<const uint4*>(wrow + 16 * sw);
+      const uint4 hi = *reinterpret_cast<const uint4*>(wrow + 16 * (sw ^ 1));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(s));
+      if (kb >= kASlots) {
+        w = mbar_wait_bounded(aempty(j), ((kb / kASlots) - 1) & 1, p.wait_limit_ns, abort_flag,
+                              p.status);
+        if (!__all_sync(0xFFFFFFFFu, w)) {
+          ok = false;
+          break;
+        }
+      }
+      uint32_t u[32];
+      unpack_word(lo.x, u + 0);
+      unpack_word(lo.y, u + 4);
+      unpack_word(lo.z, u + 8);
+      unpack_word(lo.w, u + 12);
+      unpack_word(hi.x, u + 16);
+      unpack_word(hi.y, u + 20);
+      unpack_word(hi.z, u + 24);
+      unpack_word(hi.w, u + 28);
+      tc_st_32x32b_x32(tmem + lane_addr + C::kACol0 + j * 32, u);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(afull(j));
+    }
+    if (ok) {
+      const bool w = mbar_wait_bounded(accfull, 0, p.wait_limit_ns, abort_flag, p.status);
+      ok = __all_sync(0xFFFFFFFFu, w);
+    }
+    ok = named_bar_and(1, kEpiThreads, ok);
+    if (ok) {
+      tc_fence_after();
+      int32_t* stage = reinterpret_cast<int32_t*>(s_act);   // all copies landed, all MMAs done
+      const int et = threadIdx.x - 64;                      // 0..127
+      const float beta = p.out_mode == kOutI32 ? 0.0f : *p.beta;
+      for (int c0 = 0; c0 < BN; c0 += C::kChunk) {
+        uint32_t acc[32];
+        if constexpr (C::kChunk == 32) {
+          tc_ld_32x32b_x32(tmem + lane_addr + c0, acc);
+        } else {
+          tc_ld_32x32b_x16(tmem + lane_addr + c0, acc);
+        }
+        tc_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < C::kChunk; ++jj) stage[jj * 128 + r] = static_cast<int32_t>(acc[jj]);
+        named_bar_sync(1, kEpiThreads);
+        if (!p.glu) {
+          for (int gi = et; gi < C::kChunk * 16; gi += kEpiThreads) {
+            const int jj = gi >> 4, c8 = (gi & 15) * 8;
+            const int64_t t = t0 + c0 + jj;
+            if (t >= p.T) continue;
+            const int4 a0 = *reinterpret_cast<const int4*>(stage + jj * 128 + c8);
+            const int4 a1 = *reinterpret_cast<const int4*>(stage + jj * 128 + c8 + 4);
+            const int av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const int rs = p.rowsum[t];
+            const int64_t off = t * p.ldy + r0 + c8;
+            if (p.out_mode == kOutI32) {
+              int32_t* y = reinterpret_cast<int32_t*>(p.y) + off;
+              *reinterpret_cast<int4*>(y) = make_int4(av[0] - rs, av[1] - rs, av[2] - rs, av[3] - rs);
+              *reinterpret_cast<int4*>(y + 4) = make_int4(av[4] - rs, av[5] - rs, av[6] - rs, av[7] - rs);
+            } else {
+              const float sc = __fmul_rn(__fdiv_rn(p.gamma[t], 127.0f), beta);
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = static_cast<float>(av[e] - rs) * sc;
+              if (p.out_mode == kOutF16) {
+                uint4 o;
+                __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(f[2 * e], f[2 * e + 1]);
+                *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.y) + off) = o;
+              } else {
+                float* y = reinterpret_cast<float*>(p.y) + off;
+                *reinterpret_cast<float4*>(y) = make_float4(f[0], f[1], f[2], f[3]);
+                *reinterpret_cast<float4*>(y + 4) = make_float4(f[4], f[5], f[6], f[7]);
+              }
+            }
+          }
+        } else {
+          for (int gi = et; gi < C::kChunk * 8; gi += kEpiThreads) {
+            const int jj = gi >> 3, i8 = (gi & 7) * 8;
+            const int64_t t = t0 + c0 + jj;
+            if (t >= p.T) continue;
+            const int rs = p.rowsum[t];
+            const float sc = __fmul_rn(__fdiv_rn(p.gamma[t], 127.0f), beta);
+            float hv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float yg = static_cast<float>(stage[jj * 128 + i8 + e] - rs) * sc;
+              const float yu = static_cast<float>(stage[jj * 128 + 64 + i8 + e] - rs) * sc;
+              hv[e] = sigmoid_mul(yg, yu);
+            }
+            const int64_t off = t * p.ldy + static_cast<int64_t>(blockIdx.x) * 64 + i8;
+            if (p.out_mode == kOutF16) {
+              uint4 o;
+              __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) h[e] = __floats2half2_rn(hv[2 * e], hv[2 * e + 1]);
+              *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.y) + off) = o;
+            } else {
+              float* y = reinterpret_cast<float*>(p.y) + off;
+              *reinterpret_cast<float4*>(y) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+              *reinterpret_cast<float4*>(y + 4) = make_float4(hv[4], hv[5], hv[6], hv[7]);
+            }
+          }
+        }
+        named_bar_sync(1, kEpiThreads);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmCall& c, cudaStream_t s) {
+  using Cf = Cfg<BN>;
+  static std::once_flag attr_once[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once[dev & 63], [&] {
+    attr_err = cudaFuncSetAttribute(ternary_gemm_kernel<BN>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmem);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+
+  CUtensorMap tm_w, tm_a;
+  if (!make_tmap_2d_u8(&tm_w, c.Wp, static_cast<uint64_t>(c.K / 4), static_cast<uint64_t>(c.rows),
+                       static_cast<uint64_t>(c.K / 4), kWRowBytes, 64,
+                       CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+  if (!make_tmap_2d_u8(&tm_a, c.A, static_cast<uint64_t>(c.K), static_cast<uint64_t>(c.T),
+                       static_cast<uint64_t>(c.K), kKB, BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+
+  Params p;
+  p.T = c.T;
+  p.K = c.K;
+  p.rows = c.rows;
+  p.glu = c.glu;
+  p.half = c.glu ? c.rows / 2 : 0;
+  p.out_mode = c.out_mode;
+  p.ldy = c.glu ? c.rows / 2 : c.rows;
+  p.gamma = c.gamma;
+  p.rowsum = c.rowsum;
+  p.beta = c.beta;
+  p.y = c.y;
+  p.status = c.status;
+  p.wait_limit_ns = c.wait_limit_ns;
+
+  // 128 weight rows per tile: 128 outputs, or 64 gate + 64 multiplier rows for 64 GLU outputs.
+  const unsigned ntiles = static_cast<unsigned>(c.rows / 128);
+  const unsigned ttiles = static_cast<unsigned>((c.T + BN - 1) / BN);
+  ternary_gemm_kernel<BN><<<dim3(ntiles, ttiles), kThreads, Cf::kSmem, s>>>(tm_w, tm_a, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ternary_gemm(const GemmCall& c, cudaStream_t s) {
+  if (c.T <= 16) return launch_bn<16>(c, s);
+  if (c.T <= 32) return launch_bn<32>(c, s);
+  if (c.T <= 64) return launch_bn<64>(c, s);
+  if (c.T <= 128) return launch_bn<128>(c, s);
+  return launch_bn<256>(c, s);
+}
+
+namespace {
+__global__ void wait_probe_kernel(uint64_t limit_ns, unsigned* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on this barrier: the wait must give up and report.
+    mbar_wait_bounded(smem_u32(&bar), 0, limit_ns, &abort_flag, status);
+  }
+  __syncthreads();
+}
+}  // namespace
+
+cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned* status, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(limit_ns, status);
+  return cudaGetLastError();
+}
+
+}  // namespace mmf

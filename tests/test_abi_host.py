@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every entry point
+that include/mmf.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import ternary_weight_lm_b200 as mmf
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mmf.h")
+
+OK, INVALID, SHAPE, ALIGN, CUDA, TIMEOUT, WS = 0, 1, 2, 3, 4, 5, 6
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(mmf_[a-z0-9_]+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_builds_and_loads():
+    from ternary_weight_lm_b200 import build
+    build.build()
+    assert mmf.mmf_version() == 100
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 12, names
+    L = ctypes.CDLL(mmf.lib_path)
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", mmf.lib_path], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln})
+    assert exported == names
+
+
+def test_status_strings():
+    for code, name in mmf.STATUS.items():
+        assert mmf.mmf_status_string(code) == name
+
+
+def test_workspace_sizes():
+    L = mmf.lib()
+    assert L.mmf_quantize_weights_workspace_bytes(2048, 2048) == 4096
+    # A [T x K] + gamma [T] + rowsum [T], each rounded up to 256 bytes
+    assert L.mmf_forward_workspace_bytes(64, 1024, 1024) == 64 * 1024 + 256 + 256
+    assert L.mmf_forward_workspace_bytes(3, 128, 128) == 512 + 256 + 256
+    assert L.mmf_forward_workspace_bytes(0, 128, 128) == 0
+
+
+A16 = 0x10000   # fake, aligned "device" addresses: never dereferenced by rejected calls
+
+
+def fwd(**kw):
+    a = dict(x=A16, xdt=1, T=4, K=256, g=None, eps=1e-8, Wp=A16, beta=A16, N=256, y=A16, ydt=1,
+             ws=A16, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return mmf.lib().mmf_bitlinear_forward(a["x"], a["xdt"], a["T"], a["K"], a["g"], a["eps"],
+                                           a["Wp"], a["beta"], a["N"], a["y"], a["ydt"], a["ws"],
+                                           a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), INVALID), (dict(Wp=None), INVALID), (dict(beta=None), INVALID),
+    (dict(y=None), INVALID), (dict(xdt=2), INVALID), (dict(ydt=-1), INVALID),
+    (dict(eps=0.0), INVALID), (dict(eps=-1e-8), INVALID), (dict(eps=float("nan")), INVALID),
+    (dict(T=0), SHAPE), (dict(T=-3), SHAPE), (dict(K=100), SHAPE), (dict(K=64), SHAPE),
+    (dict(K=8320), SHAPE), (dict(N=192), SHAPE), (dict(N=0), SHAPE),
+    (dict(x=A16 + 8), ALIGN), (dict(y=A16 + 2), ALIGN), (dict(Wp=A16 + 4), ALIGN),
+    (dict(g=A16 + 4), ALIGN), (dict(ws=A16 + 16), ALIGN),
+    (dict(ws=None), WS), (dict(wsb=100), WS),
+])
+def test_forward_rejects_on_host(kw, code):
+    assert fwd(**kw) == code
+
+
+def test_glu_and_other_entry_points_reject_on_host():
+    L = mmf.lib()
+    # N2 must be a multiple of 128 (so that I is a multiple of 64)
+    assert L.mmf_bitlinear_glu_forward(A16, 1, 4, 256, None, 1e-8, A16, A16, 192, A16, 1, A16,
+                                       1 << 20, None) == SHAPE
+    assert L.mmf_quantize_weights(None, 0, 128, 128, A16, A16, A16, 4096, None) == INVALID
+    assert L.mmf_quantize_weights(A16, 0, 128, 120, A16, A16, A16, 4096, None) == SHAPE
+    assert L.mmf_quantize_weights(A16, 0, 128, 128, A16, A16, A16, 100, None) == WS
+    assert L.mmf_quantize_weights(A16 + 4, 0, 128, 128, A16, A16, A16, 4096, None) == ALIGN
+    assert L.mmf_ternary_encode(A16, 5, 128, 128, A16, A16, None) == INVALID
+    assert L.mmf_quantize_activations(A16, 1, 4, 256, None, 0.0, A16, A16, None, None) == INVALID
+    assert L.mmf_quantize_activations(A16, 1, 4, 200, None, 1e-8, A16, A16, None, None) == SHAPE
+    assert L.mmf_ternary_accumulate_i32(A16, 4, 256, A16, 256, A16 + 4, A16, 1 << 20,
+                                        None) == ALIGN
+    assert L.mmf_ternary_accumulate_i32(A16, 4, 256, A16, 256, A16, A16, 10, None) == WS
+    assert L.mmf_debug_wait_timeout_probe(10, None) == INVALID
+    assert L.mmf_debug_wait_timeout_probe(10 ** 10, None) == INVALID
+
+
+def test_valid_call_without_gpu_reports_cuda_error():
+    # With no CUDA device the call must fail loudly (no host fallback exists).
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert fwd() == CUDA
+    with pytest.raises(mmf.MMFError):
+        mmf._check("mmf_bitlinear_forward", fwd())
