@@ -122,6 +122,15 @@ mmf_status mmf_quantize_activations(const void* x, mmf_dtype xdt, int64_t T, int
                                     const float* norm_w, float eps, int8_t* A, float* gamma,
                                     int32_t* rowsum, void* stream);
 
+/* Second half of the forward: contraction + dequantisation (+ SiLU-GLU when glu != 0, then
+ * N is 2I and y is T x I) from activation codes already produced by mmf_quantize_activations
+ * (A [T x K], gamma [T], rowsum [T]).  One launch.  Lets callers reuse one quantised input
+ * for several projections whose norm weights are equal. */
+mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const float* gamma,
+                                           const int32_t* rowsum, int64_t T, int64_t K,
+                                           const uint8_t* Wp, const float* beta, int64_t N,
+                                           int glu, void* y, mmf_dtype ydt, void* stream);
+
 /* acc [T x N] int32 = ternary accumulation of given codes A [T x K] against Wp.  Exact.
  * ws must hold mmf_forward_workspace_bytes(T, K, N). */
 mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int64_t K, const uint8_t* Wp,

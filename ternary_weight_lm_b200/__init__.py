@@ -17,7 +17,8 @@ __all__ = [
     "MMFError", "lib", "lib_path",
     "mmf_quantize_weights_workspace_bytes", "mmf_quantize_weights", "mmf_ternary_encode",
     "mmf_forward_workspace_bytes", "mmf_bitlinear_forward", "mmf_bitlinear_glu_forward",
-    "mmf_quantize_activations", "mmf_ternary_accumulate_i32", "mmf_get_device_status",
+    "mmf_quantize_activations", "mmf_bitlinear_forward_quantized",
+    "mmf_ternary_accumulate_i32", "mmf_get_device_status",
     "mmf_debug_wait_timeout_probe", "mmf_status_string", "mmf_version",
     "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
     "MMF_F32", "MMF_F16", "STATUS",
@@ -60,6 +61,7 @@ def lib():
             "mmf_bitlinear_forward": ([P, I, I64, I64, P, F, P, P, I64, P, I, P, SZ, P], I),
             "mmf_bitlinear_glu_forward": ([P, I, I64, I64, P, F, P, P, I64, P, I, P, SZ, P], I),
             "mmf_quantize_activations": ([P, I, I64, I64, P, F, P, P, P, P], I),
+            "mmf_bitlinear_forward_quantized": ([P, P, P, I64, I64, P, P, I64, I, P, I, P], I),
             "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
             "mmf_get_device_status": ([], I),
             "mmf_debug_wait_timeout_probe": ([ctypes.c_uint64, P], I),
@@ -150,6 +152,13 @@ def mmf_quantize_activations(x, norm_w, eps, A, gamma, rowsum=None, stream=None)
     _check("mmf_quantize_activations", lib().mmf_quantize_activations(
         _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(A), _ptr(gamma), _ptr(rowsum),
         _stream(stream)))
+
+
+def mmf_bitlinear_forward_quantized(A, gamma, rowsum, Wp, beta, N, glu, y, stream=None):
+    T, K = A.shape
+    _check("mmf_bitlinear_forward_quantized", lib().mmf_bitlinear_forward_quantized(
+        _ptr(A), _ptr(gamma), _ptr(rowsum), T, K, _ptr(Wp), _ptr(beta), N, 1 if glu else 0,
+        _ptr(y), _dt(y), _stream(stream)))
 
 
 def mmf_ternary_accumulate_i32(A, Wp, N, acc, ws, stream=None):

@@ -226,6 +226,38 @@ MMF_EXPORT mmf_status mmf_quantize_activations(const void* x, mmf_dtype xdt, int
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
+MMF_EXPORT mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const float* gamma,
+                                                      const int32_t* rowsum, int64_t T, int64_t K,
+                                                      const uint8_t* Wp, const float* beta,
+                                                      int64_t N, int glu, void* y, mmf_dtype ydt,
+                                                      void* stream) {
+  if (!A || !gamma || !rowsum || !Wp || !beta || !y) return MMF_ERR_INVALID_ARG;
+  if (check_dtype(ydt) != MMF_OK || (glu != 0 && glu != 1)) return MMF_ERR_INVALID_ARG;
+  mmf_status st;
+  if ((st = check_t(T)) != MMF_OK || (st = check_k(K)) != MMF_OK || (st = check_n(N)) != MMF_OK)
+    return st;
+  if (!aligned(A, 16) || !aligned(Wp, 16) || !aligned(y, 16) || !aligned(gamma, 4) ||
+      !aligned(rowsum, 4) || !aligned(beta, 4))
+    return MMF_ERR_ALIGNMENT;
+  unsigned* status = status_ptr();
+  if (!status) return MMF_ERR_CUDA;
+  GemmCall c;
+  c.A = A;
+  c.Wp = Wp;
+  c.T = T;
+  c.K = static_cast<int>(K);
+  c.rows = static_cast<int>(N);
+  c.glu = glu;
+  c.gamma = gamma;
+  c.rowsum = rowsum;
+  c.beta = beta;
+  c.y = y;
+  c.out_mode = ydt == MMF_F16 ? kOutF16 : kOutF32;
+  c.status = status;
+  c.wait_limit_ns = kWaitLimitNs;
+  return from_cuda(launch_ternary_gemm(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 MMF_EXPORT mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int64_t K,
                                                  const uint8_t* Wp, int64_t N, int32_t* acc,
                                                  void* ws, size_t ws_bytes, void* stream) {
