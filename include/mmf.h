@@ -137,6 +137,25 @@ mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int64_t K, con
                                       int64_t N, int32_t* acc, void* ws, size_t ws_bytes,
                                       void* stream);
 
+/* ---- forward without any allocation ------------------------------------------------------ */
+
+/* The pages have no counterpart to this entry point; it serves callers that cannot call
+ * cudaMalloc (a plugin inside an application that owns all device memory, a real-time decode
+ * loop that must not allocate, C code without a device allocator).  Same arguments and
+ * result as mmf_bitlinear_forward, without the workspace: the scratch (int8 codes [T x K],
+ * gamma [T], code sums [T], each rounded up to 256 bytes) lives in a fixed 4 MiB device
+ * array that every GPU loading the library holds until the process exits.  Calls whose
+ * scratch would exceed 4 MiB are rejected with MMF_ERR_WORKSPACE before any launch (for
+ * example T = 64 with K = 8192 fits; T = 512 with K = 8192 does not).  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, device current); make
+ * that first call before any stream capture.  All calls share the array: nothing in it needs
+ * to start at zero, but calls whose work overlaps on the GPU race on it, so order them on one
+ * stream (or with events). */
+mmf_status mmf_bitlinear_forward_noalloc(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
+                                         const float* norm_w, float eps, const uint8_t* Wp,
+                                         const float* beta, int64_t N, void* y, mmf_dtype ydt,
+                                         void* stream);
+
 /* ---- status ------------------------------------------------------------------------------ */
 
 /* Reads and clears the device status word of the current device (synchronises the device).

@@ -18,7 +18,7 @@ __all__ = [
     "mmf_quantize_weights_workspace_bytes", "mmf_quantize_weights", "mmf_ternary_encode",
     "mmf_forward_workspace_bytes", "mmf_bitlinear_forward", "mmf_bitlinear_glu_forward",
     "mmf_quantize_activations", "mmf_bitlinear_forward_quantized",
-    "mmf_ternary_accumulate_i32", "mmf_get_device_status",
+    "mmf_ternary_accumulate_i32", "mmf_bitlinear_forward_noalloc", "mmf_get_device_status",
     "mmf_debug_wait_timeout_probe", "mmf_status_string", "mmf_version",
     "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
     "MMF_F32", "MMF_F16", "STATUS",
@@ -63,6 +63,7 @@ def lib():
             "mmf_quantize_activations": ([P, I, I64, I64, P, F, P, P, P, P], I),
             "mmf_bitlinear_forward_quantized": ([P, P, P, I64, I64, P, P, I64, I, P, I, P], I),
             "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
+            "mmf_bitlinear_forward_noalloc": ([P, I, I64, I64, P, F, P, P, I64, P, I, P], I),
             "mmf_get_device_status": ([], I),
             "mmf_debug_wait_timeout_probe": ([ctypes.c_uint64, P], I),
             "mmf_status_string": ([I], ctypes.c_char_p),
@@ -165,6 +166,15 @@ def mmf_ternary_accumulate_i32(A, Wp, N, acc, ws, stream=None):
     T, K = A.shape
     _check("mmf_ternary_accumulate_i32", lib().mmf_ternary_accumulate_i32(
         _ptr(A), T, K, _ptr(Wp), N, _ptr(acc), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def mmf_bitlinear_forward_noalloc(x, norm_w, eps, Wp, beta, N, y, stream=None):
+    """Forward without a workspace argument: for callers that cannot allocate device memory.
+    Scratch is a fixed 4 MiB device array shared by all calls (see include/mmf.h)."""
+    T, K = x.shape
+    _check("mmf_bitlinear_forward_noalloc", lib().mmf_bitlinear_forward_noalloc(
+        _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(Wp), _ptr(beta), N, _ptr(y),
+        _dt(y), _stream(stream)))
 
 
 def mmf_get_device_status():

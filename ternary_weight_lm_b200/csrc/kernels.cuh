@@ -46,6 +46,9 @@ struct GemmCall {
 };
 cudaError_t launch_ternary_gemm(const GemmCall& c, cudaStream_t s);
 
+// Device address of the library's status word on the current device (nullptr on failure).
+unsigned* device_status_word();
+
 // One block, one wait that nothing satisfies: must give up after limit_ns.
 cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned* status, cudaStream_t s);
 

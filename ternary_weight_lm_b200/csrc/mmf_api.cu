@@ -136,6 +136,8 @@ mmf_status fwd_common(const void* x, int xdt, int64_t T, int64_t K, const float*
 
 }  // namespace
 
+unsigned* device_status_word() { return status_ptr(); }
+
 bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                      CUtensorMapSwizzle swz) {
