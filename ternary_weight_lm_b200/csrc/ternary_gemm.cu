@@ -35,7 +35,6 @@ constexpr int kKB = 128;                       // K elements per pipeline stage
 constexpr int kWRowBytes = kKB / 4;            // packed bytes of one weight row per stage
 constexpr int kWHalfBytes = 64 * kWRowBytes;   // one TMA box: 64 rows x 32 bytes
 constexpr int kWStageBytes = 2 * kWHalfBytes;  // 128 rows
-constexpr int kASlots = 4;                     // TMEM slots of unpacked weights (32 columns)
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint64_t kDrainNs = 2000000000ull;
@@ -44,16 +43,22 @@ template <int BN>
 struct Cfg {
   static constexpr int kActStage = BN * kKB;               // int8 activation tile
   static constexpr int kStage = kActStage + kWStageBytes;
-  static constexpr int kStagesRaw = (200 * 1024) / kStage;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kTmemCols = BN <= 128 ? 256 : 512;
-  static constexpr int kACol0 = BN <= 128 ? 128 : 256;     // first TMEM column of A slots
+  // One ring: stage s of shared memory and slot s of TMEM (the unpacked weights of that
+  // stage) are filled and freed together, so every role waits on one barrier per k-block.
+  static constexpr int kTmemCols = 512;                    // one CTA per SM owns all of TMEM
+  static constexpr int kACol0 = ((BN + 31) / 32) * 32;     // first TMEM column of A slots
+  static constexpr int kSlotsMax = (kTmemCols - kACol0) / 32;
+  static constexpr int kStagesSmem = (214 * 1024) / kStage;
+  static constexpr int kS0 = kStagesSmem < kSlotsMax ? kStagesSmem : kSlotsMax;
+  static constexpr int kStages = kS0 > 16 ? 16 : kS0;
   static constexpr int kChunk = BN < 32 ? BN : 32;         // epilogue token columns per pass
-  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kASlots + 1);
-  // Request at least ~116 KB so only one CTA lives on an SM (its TMEM allocation never waits).
-  static constexpr int kSmemUsed = 1024 + kStages * kStage + kBarBytes;
+  static constexpr int kBarBytes = 8 * (3 * kStages + 1);
+  static constexpr int kTokBytes = 8 * BN;                 // per-token scale and code sum
+  static constexpr int kSmemUsed = 1024 + kStages * kStage + kBarBytes + kTokBytes;
+  // At least ~116 KB so only one CTA lives on an SM (its TMEM allocation never waits).
   static constexpr int kSmem = kSmemUsed < 118 * 1024 ? 118 * 1024 : kSmemUsed;
-  static_assert(kStages >= 2, "pipeline needs two stages");
+  static_assert(kStages >= 4, "pipeline needs four stages");
+  static_assert(kSmem <= 227 * 1024, "shared memory per block");
   static_assert(kChunk * 128 * 4 <= kStages * kActStage, "epilogue staging must fit");
 };
 
@@ -96,6 +101,8 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   uint8_t* s_act = smem;
   uint8_t* s_w = smem + C::kStages * C::kActStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + C::kStages * kWStageBytes);
+  float* s_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::kBarBytes);
+  int32_t* s_rsum = reinterpret_cast<int32_t*>(s_scale + BN);
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -111,20 +118,19 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     r1 = r0 + 64;
   }
 
+  // full(s): the stage's TMA bytes landed.  afull(s): the four unpack warps wrote TMEM slot s
+  // (they did so after seeing full(s), so afull(s) also implies the activation tile is in).
+  // empty(s): the MMAs of the stage completed and the unpack warps read its packed weights.
   auto full = [&](int s) { return smem_u32(bars + s); };
-  auto empty = [&](int s) { return smem_u32(bars + C::kStages + s); };
-  auto afull = [&](int j) { return smem_u32(bars + 2 * C::kStages + j); };
-  auto aempty = [&](int j) { return smem_u32(bars + 2 * C::kStages + kASlots + j); };
-  const uint32_t accfull = smem_u32(bars + 2 * C::kStages + 2 * kASlots);
+  auto afull = [&](int s) { return smem_u32(bars + C::kStages + s); };
+  auto empty = [&](int s) { return smem_u32(bars + 2 * C::kStages + s); };
+  const uint32_t accfull = smem_u32(bars + 3 * C::kStages);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full(s), 1);
+      mbar_init(afull(s), 4);       // the four unpack warps
       mbar_init(empty(s), 1 + 4);   // the MMA commit + the four unpack warps
-    }
-    for (int j = 0; j < kASlots; ++j) {
-      mbar_init(afull(j), 4);
-      mbar_init(aempty(j), 1);
     }
     mbar_init(accfull, 1);
     s_abort = 0;
@@ -173,23 +179,25 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
+      const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
+      int s = 0;
+      uint32_t ph = 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % C::kStages, j = kb % kASlots;
-        if (!mbar_wait_bounded(full(s), (kb / C::kStages) & 1, p.wait_limit_ns, abort_flag,
-                               p.status))
-          break;
-        if (!mbar_wait_bounded(afull(j), (kb / kASlots) & 1, p.wait_limit_ns, abort_flag,
-                               p.status))
-          break;
+        if (!mbar_wait_bounded(afull(s), ph, p.wait_limit_ns, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t b0 = smem_u32(s_act + s * C::kActStage);
-#pragma unroll
-        for (int kk = 0; kk < kKB / 32; ++kk) {
-          tc_mma_i8_ts(tmem, tmem + C::kACol0 + j * 32 + kk * 8, smem_desc_kmajor_sw128(b0 + kk * 32),
-                       idesc, (kb | kk) != 0 ? 1u : 0u);
-        }
+        // descriptor start address is in 16-byte units: a stage is kActStage bytes, a 32-deep
+        // k step is 32 bytes within the 128-byte swizzled rows
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kActStage) >> 4);
+        const uint32_t ad = tmem + C::kACol0 + s * 32;
+        tc_mma_i8_ts(tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
+        tc_mma_i8_ts(tmem, ad + 8, bd + 2, idesc, 1u);
+        tc_mma_i8_ts(tmem, ad + 16, bd + 4, idesc, 1u);
+        tc_mma_i8_ts(tmem, ad + 24, bd + 6, idesc, 1u);
         tc_commit(empty(s));
-        tc_commit(aempty(j));
+        if (++s == C::kStages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
       // Signals the epilogue; in the abort path it also tells this thread when the MMAs it
       // issued have finished, so TMEM is not freed under them.
@@ -203,11 +211,29 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
     // Wait outcomes are made warp-uniform (__all_sync) before the .sync.aligned tcgen05
     // instructions, and the epilogue is entered by all four warps or by none.
+    // Per-token dequantisation scale (gamma/127 * beta) and code sum for this tile, staged
+    // once so the epilogue does no dependent global loads.
+    if (p.out_mode != kOutI32) {
+      const float beta = *p.beta;
+      for (int i = threadIdx.x - 64; i < BN; i += kEpiThreads) {
+        const int64_t t = t0 + i;
+        s_scale[i] = t < p.T ? __fmul_rn(__fdiv_rn(p.gamma[t], 127.0f), beta) : 0.0f;
+        s_rsum[i] = t < p.T ? p.rowsum[t] : 0;
+      }
+    } else {
+      for (int i = threadIdx.x - 64; i < BN; i += kEpiThreads) {
+        const int64_t t = t0 + i;
+        s_scale[i] = 0.0f;
+        s_rsum[i] = t < p.T ? p.rowsum[t] : 0;
+      }
+    }
     bool ok = true;
+    int s = 0;
+    uint32_t ph = 0;
     for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % C::kStages, j = kb % kASlots;
-      bool w = mbar_wait_bounded(full(s), (kb / C::kStages) & 1, p.wait_limit_ns, abort_flag,
-                                 p.status);
+      // full(s) of this use implies the previous use of stage s was released (the producer
+      // waited for it before reloading), so TMEM slot s is free as well.
+      const bool w = mbar_wait_bounded(full(s), ph, p.wait_limit_ns, abort_flag, p.status);
       if (!__all_sync(0xFFFFFFFFu, w)) {
         ok = false;
         break;
@@ -219,14 +245,6 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       const uint4 hi = *reinterpret_cast<const uint4*>(wrow + 16 * (sw ^ 1));
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
-      if (kb >= kASlots) {
-        w = mbar_wait_bounded(aempty(j), ((kb / kASlots) - 1) & 1, p.wait_limit_ns, abort_flag,
-                              p.status);
-        if (!__all_sync(0xFFFFFFFFu, w)) {
-          ok = false;
-          break;
-        }
-      }
       uint32_t u[32];
       unpack_word(lo.x, u + 0);
       unpack_word(lo.y, u + 4);
@@ -236,11 +254,15 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       unpack_word(hi.y, u + 20);
       unpack_word(hi.z, u + 24);
       unpack_word(hi.w, u + 28);
-      tc_st_32x32b_x32(tmem + lane_addr + C::kACol0 + j * 32, u);
+      tc_st_32x32b_x32(tmem + lane_addr + C::kACol0 + s * 32, u);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(afull(j));
+      if (lane == 0) mbar_arrive(afull(s));
+      if (++s == C::kStages) {
+        s = 0;
+        ph ^= 1u;
+      }
     }
     if (ok) {
       const bool w = mbar_wait_bounded(accfull, 0, p.wait_limit_ns, abort_flag, p.status);
@@ -251,7 +273,6 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       tc_fence_after();
       int32_t* stage = reinterpret_cast<int32_t*>(s_act);   // all copies landed, all MMAs done
       const int et = threadIdx.x - 64;                      // 0..127
-      const float beta = p.out_mode == kOutI32 ? 0.0f : *p.beta;
       for (int c0 = 0; c0 < BN; c0 += C::kChunk) {
         uint32_t acc[32];
         if constexpr (C::kChunk == 32) {
@@ -271,14 +292,14 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
             const int4 a0 = *reinterpret_cast<const int4*>(stage + jj * 128 + c8);
             const int4 a1 = *reinterpret_cast<const int4*>(stage + jj * 128 + c8 + 4);
             const int av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const int rs = p.rowsum[t];
+            const int rs = s_rsum[c0 + jj];
             const int64_t off = t * p.ldy + r0 + c8;
             if (p.out_mode == kOutI32) {
               int32_t* y = reinterpret_cast<int32_t*>(p.y) + off;
               *reinterpret_cast<int4*>(y) = make_int4(av[0] - rs, av[1] - rs, av[2] - rs, av[3] - rs);
               *reinterpret_cast<int4*>(y + 4) = make_int4(av[4] - rs, av[5] - rs, av[6] - rs, av[7] - rs);
             } else {
-              const float sc = __fmul_rn(__fdiv_rn(p.gamma[t], 127.0f), beta);
+              const float sc = s_scale[c0 + jj];
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = static_cast<float>(av[e] - rs) * sc;
@@ -300,8 +321,8 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
             const int jj = gi >> 3, i8 = (gi & 7) * 8;
             const int64_t t = t0 + c0 + jj;
             if (t >= p.T) continue;
-            const int rs = p.rowsum[t];
-            const float sc = __fmul_rn(__fdiv_rn(p.gamma[t], 127.0f), beta);
+            const int rs = s_rsum[c0 + jj];
+            const float sc = s_scale[c0 + jj];
             float hv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
