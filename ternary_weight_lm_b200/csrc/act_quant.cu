@@ -106,6 +106,10 @@ act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, 
   const int64_t row = blockIdx.x;
   const int nvec = K / E;
   const TIn* xr = x + row * static_cast<int64_t>(K);
+  // The next launch may begin its set-up; this grid waits for its own producers before it
+  // reads x (which the previous launch may have written).
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   float v[MAXV][E];
   double ss = 0.0;
@@ -207,17 +211,23 @@ rowsum_kernel(const int8_t* __restrict__ A, int K, int32_t* __restrict__ rowsum)
 
 cudaError_t launch_act_quant(const void* x, int xdt, int64_t T, int K, const float* g, float eps,
                              int8_t* A, float* gamma, int32_t* rowsum, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(T));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(T));
+  cfg.blockDim = dim3(kAqThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
   if (xdt == kInF16) {
     // 8 halves per vector: K <= 128 * 8 * 8 = 8192
-    act_quant_kernel<__half, 8><<<grid, kAqThreads, 0, s>>>(
-        reinterpret_cast<const __half*>(x), K, g, eps, A, gamma, rowsum);
-  } else {
-    // 4 floats per vector: K <= 128 * 16 * 4 = 8192
-    act_quant_kernel<float, 16><<<grid, kAqThreads, 0, s>>>(
-        reinterpret_cast<const float*>(x), K, g, eps, A, gamma, rowsum);
+    return cudaLaunchKernelEx(&cfg, act_quant_kernel<__half, 8>,
+                              reinterpret_cast<const __half*>(x), K, g, eps, A, gamma, rowsum);
   }
-  return cudaGetLastError();
+  // 4 floats per vector: K <= 128 * 16 * 4 = 8192
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<float, 16>,
+                            reinterpret_cast<const float*>(x), K, g, eps, A, gamma, rowsum);
 }
 
 cudaError_t launch_rowsum(const int8_t* A, int64_t T, int K, int32_t* rowsum, cudaStream_t s) {

@@ -38,6 +38,7 @@ constexpr int kWStageBytes = 2 * kWHalfBytes;  // 128 rows
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr uint64_t kDrainNs = 2000000000ull;
+constexpr int64_t kSplitTargetCtas = 148;       // SMs of a B200
 
 template <int BN>
 struct Cfg {
@@ -90,6 +91,54 @@ __device__ __forceinline__ float sigmoid_mul(float g, float u) {
   return __fdividef(g, 1.0f + expf(-g)) * u;
 }
 
+// Split-K epilogue: CTA z of the cluster finalises tokens [z*BN/C, (z+1)*BN/C) of the tile,
+// adding the C partial sums (exact int32) read from each CTA's shared memory.  Thread et is
+// tile row et (non-GLU) or output column et < 64 (GLU: row et is the gated half, row et + 64
+// the multiplier).
+template <int BN>
+__device__ __forceinline__ void split_k_reduce(const Params& p, int csize, int64_t t0, int r0,
+                                               const uint8_t* s_act, const float* s_scale,
+                                               const int32_t* s_rsum) {
+  const int et = threadIdx.x - 64;
+  const uint32_t crank = cluster_ctarank();
+  const int per = BN / csize;
+  const uint32_t part0 = smem_u32(s_act);
+  for (int j = static_cast<int>(crank) * per; j < (static_cast<int>(crank) + 1) * per; ++j) {
+    const int64_t t = t0 + j;
+    if (t >= p.T) break;
+    if (!p.glu) {
+      int32_t v = 0;
+      for (int c = 0; c < csize; ++c)
+        v += ld_cluster_s32(map_peer(part0 + 4u * static_cast<uint32_t>(j * 128 + et), c));
+      v -= s_rsum[j];
+      const int64_t off = t * p.ldy + r0 + et;
+      if (p.out_mode == kOutI32) {
+        reinterpret_cast<int32_t*>(p.y)[off] = v;
+      } else {
+        const float f = static_cast<float>(v) * s_scale[j];
+        if (p.out_mode == kOutF16)
+          reinterpret_cast<__half*>(p.y)[off] = __float2half_rn(f);
+        else
+          reinterpret_cast<float*>(p.y)[off] = f;
+      }
+    } else if (et < 64) {
+      int32_t g = 0, u = 0;
+      for (int c = 0; c < csize; ++c) {
+        g += ld_cluster_s32(map_peer(part0 + 4u * static_cast<uint32_t>(j * 128 + et), c));
+        u += ld_cluster_s32(map_peer(part0 + 4u * static_cast<uint32_t>(j * 128 + 64 + et), c));
+      }
+      const float yg = static_cast<float>(g - s_rsum[j]) * s_scale[j];
+      const float yu = static_cast<float>(u - s_rsum[j]) * s_scale[j];
+      const float h = sigmoid_mul(yg, yu);
+      const int64_t off = t * p.ldy + static_cast<int64_t>(blockIdx.x) * 64 + et;
+      if (p.out_mode == kOutF16)
+        reinterpret_cast<__half*>(p.y)[off] = __float2half_rn(h);
+      else
+        reinterpret_cast<float*>(p.y)[off] = h;
+    }
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
@@ -107,7 +156,12 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   __shared__ int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nkb = p.K / kKB;
+  // Split K: the gridDim.z CTAs of a cluster share one output tile and each sums a contiguous
+  // range of k-blocks; their int32 partial sums are added through distributed shared memory.
+  const int csize = static_cast<int>(gridDim.z);
+  const int nkb_all = p.K / kKB;
+  const int kb0 = static_cast<int>(blockIdx.z) * nkb_all / csize;
+  const int nkb = (static_cast<int>(blockIdx.z) + 1) * nkb_all / csize - kb0;
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * BN;
   int r0, r1;  // first weight row of each 64-row half of the tile
   if (p.glu) {
@@ -149,6 +203,11 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
+  // Everything above is private set-up.  From here on the kernel reads and writes global
+  // memory, so it first waits for the launches it depends on; the next launch may begin its
+  // own set-up now.
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -162,12 +221,13 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
             !mbar_wait_bounded(empty(s), ((kb / C::kStages) - 1) & 1, p.wait_limit_ns,
                                abort_flag, p.status))
           break;
+        const int kg = kb0 + kb;   // k-block index within the whole K
         mbar_arrive_expect_tx(full(s), C::kStage);
-        tma_load_2d(smem_u32(s_act + s * C::kActStage), &tm_a, full(s), kb * kKB,
+        tma_load_2d(smem_u32(s_act + s * C::kActStage), &tm_a, full(s), kg * kKB,
                     static_cast<int32_t>(t0), pol_a);
         uint8_t* wdst = s_w + s * kWStageBytes;
-        tma_load_2d(smem_u32(wdst), &tm_w, full(s), kb * kWRowBytes, r0, pol_w);
-        tma_load_2d(smem_u32(wdst + kWHalfBytes), &tm_w, full(s), kb * kWRowBytes, r1, pol_w);
+        tma_load_2d(smem_u32(wdst), &tm_w, full(s), kg * kWRowBytes, r0, pol_w);
+        tma_load_2d(smem_u32(wdst + kWHalfBytes), &tm_w, full(s), kg * kWRowBytes, r1, pol_w);
         issued = kb + 1;
       }
       // Every copy this thread started must land before the block may exit.
@@ -189,7 +249,7 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
         // k step is 32 bytes within the 128-byte swizzled rows
         const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kActStage) >> 4);
         const uint32_t ad = tmem + C::kACol0 + s * 32;
-        tc_mma_i8_ts(tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);
+        tc_mma_i8_ts(tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);   // kb counts this CTA's range
         tc_mma_i8_ts(tmem, ad + 8, bd + 2, idesc, 1u);
         tc_mma_i8_ts(tmem, ad + 16, bd + 4, idesc, 1u);
         tc_mma_i8_ts(tmem, ad + 24, bd + 6, idesc, 1u);
@@ -269,7 +329,23 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       ok = __all_sync(0xFFFFFFFFu, w);
     }
     ok = named_bar_and(1, kEpiThreads, ok);
-    if (ok) {
+    if (ok && csize > 1) {
+      // Split K: dump this CTA's partial sums to shared memory as int32 [token][row]; the
+      // cluster adds them after the cluster barrier below.
+      tc_fence_after();
+      int32_t* part = reinterpret_cast<int32_t*>(s_act);
+      for (int c0 = 0; c0 < BN; c0 += C::kChunk) {
+        uint32_t acc[32];
+        if constexpr (C::kChunk == 32) {
+          tc_ld_32x32b_x32(tmem + lane_addr + c0, acc);
+        } else {
+          tc_ld_32x32b_x16(tmem + lane_addr + c0, acc);
+        }
+        tc_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < C::kChunk; ++jj) part[(c0 + jj) * 128 + r] = static_cast<int32_t>(acc[jj]);
+      }
+    } else if (ok) {
       tc_fence_after();
       int32_t* stage = reinterpret_cast<int32_t*>(s_act);   // all copies landed, all MMAs done
       const int et = threadIdx.x - 64;                      // 0..127
@@ -351,6 +427,12 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
 
   tc_fence_before();
   __syncthreads();
+  if (csize > 1) {
+    // Every thread of every CTA of the cluster reaches both barriers on every path.
+    cluster_sync_all();
+    if (warp >= 2) split_k_reduce<BN>(p, csize, t0, r0, s_act, s_scale, s_rsum);
+    cluster_sync_all();   // peers' partial sums stay readable until everyone is done
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -399,8 +481,30 @@ cudaError_t launch_bn(const GemmCall& c, cudaStream_t s) {
   // 128 weight rows per tile: 128 outputs, or 64 gate + 64 multiplier rows for 64 GLU outputs.
   const unsigned ntiles = static_cast<unsigned>(c.rows / 128);
   const unsigned ttiles = static_cast<unsigned>((c.T + BN - 1) / BN);
-  ternary_gemm_kernel<BN><<<dim3(ntiles, ttiles), kThreads, Cf::kSmem, s>>>(tm_w, tm_a, p);
-  return cudaGetLastError();
+  // Few tiles (decode): split K over a cluster of up to 8 CTAs so more SMs stream weights.
+  const int nkb = c.K / kKB;
+  const int64_t tiles = static_cast<int64_t>(ntiles) * ttiles;
+  int csize = 1;
+  if (tiles < kSplitTargetCtas) {
+    const int64_t room = kSplitTargetCtas / tiles;
+    while (csize * 2 <= 8 && csize * 2 <= nkb && csize * 2 <= room) csize *= 2;
+  }
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ntiles, ttiles, static_cast<unsigned>(csize));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cf::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  attrs[1].id = cudaLaunchAttributeClusterDimension;
+  attrs[1].val.clusterDim.x = 1;
+  attrs[1].val.clusterDim.y = 1;
+  attrs[1].val.clusterDim.z = static_cast<unsigned>(csize);
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, ternary_gemm_kernel<BN>, tm_w, tm_a, p);
 }
 
 }  // namespace
