@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target host time of the CPU-baseline sample")
+    ap.add_argument("--path", choices=["auto", "program", "launches"], default="auto",
+                    help="one program launch per step (decode, T <= 64) or per-projection launches")
     return ap.parse_args(argv)
 
 
@@ -187,91 +189,147 @@ def quant_bytes(p, T, in_bytes=2):
     return in_bytes * T * p.K + T * p.K + 8 * T
 
 
-class GpuWorkload:
-    """Device buffers for one replica: packed weight copies, inputs, outputs, workspaces."""
+def step_bytes(wl):
+    """Algorithmic HBM bytes of one step run as one program launch: every projection's packed
+    weights, its input read once (fp16) and its output written once; the int8 codes are an
+    on-chip/L2 intermediate."""
+    T, tot = wl.T, 0
+    for p in wl.projections:
+        n_out = p.N // 2 if p.glu else p.N
+        tot += p.N * p.K // 4 + 2 * T * p.K + 2 * T * n_out
+    return tot * wl.layers
 
-    def __init__(self, wl, device, copies=None):
+
+# Data flow of one layer, in dependency order: i/f/g read the layer input; o reads g's output
+# (standing in for the recurrence output); gate reads o's output (standing in for the residual
+# and norm); down reads the GLU output; the next layer reads down's output.
+LEVEL_OF = {"i_proj": 0, "f_proj": 0, "g_proj": 0, "o_proj": 1, "gate_proj": 2, "down_proj": 3,
+            "proj": 0}
+
+
+class GpuWorkload:
+    """Device buffers for one replica: packed weight copies, the step input, per-layer outputs,
+    and either one planned program per weight copy (T <= 64) or per-projection launches."""
+
+    def __init__(self, wl, device, path="auto"):
         import torch
         import ternary_weight_lm_b200 as mmf
         self.torch, self.mmf = torch, mmf
         self.wl, self.dev = wl, device
         T = wl.T
         H = wl.projections[0].K
-        layer_bytes = wl.packed_bytes_per_layer
-        if copies is None:
-            need = 2 * L2_BYTES
-            copies = max(1, -(-need // (layer_bytes * wl.layers)))
-        self.copies = copies
-        self.n_layers_total = copies * wl.layers
-        xdt = torch.float32 if wl.x_dtype == "f32" else torch.float16
+        need = 2 * L2_BYTES
+        self.copies = max(1, -(-need // (wl.packed_bytes_per_layer * wl.layers)))
+        xdt = np.float32 if wl.x_dtype == "f32" else np.float16
         self.ydt = torch.float32 if wl.y_dtype == "f32" else torch.float16
-        # one seeded layer, quantised by the library; every other layer is a byte copy at a
-        # distinct address (identical bytes stream the same as distinct ones)
+        # one seeded layer quantised by the library; every other layer and copy is a byte copy at
+        # a distinct address (identical bytes stream exactly like distinct ones)
         self.Wp, self.beta = {}, {}
         for p in wl.projections:
             W = torch.from_numpy(synth.weights(0, p.name, p.N, p.K)).to(device)
             Wp0, b0 = mmf.quantize_weights(W)
             del W
-            self.Wp[p.name] = [Wp0] + [Wp0.clone() for _ in range(self.n_layers_total - 1)]
-            self.beta[p.name] = [b0] + [b0.clone() for _ in range(self.n_layers_total - 1)]
-        srcs = sorted({p.src for p in wl.projections if p.src != "h"})
-        self.x = {s: torch.from_numpy(synth.activations(0, s, T, H, dtype=np.float16
-                                                         if xdt == torch.float16 else np.float32,
-                                                         outlier_frac=wl.outlier_frac,
-                                                         outlier_scale=wl.outlier_scale)
-                                      ).to(device) for s in srcs}
-        self.y = {}
-        for p in wl.projections:
-            n_out = p.N // 2 if p.glu else p.N
-            self.y[p.name] = torch.empty((T, n_out), dtype=self.ydt, device=device)
-        kmax = max(p.K for p in wl.projections)
-        nmax = max(p.N for p in wl.projections)
-        self.ws = mmf.workspace(mmf.mmf_forward_workspace_bytes(T, kmax, nmax), device)
-        # split buffers for the instrumented pass
-        self.A = torch.empty((T, kmax), dtype=torch.int8, device=device)
-        self.gamma = torch.empty(T, dtype=torch.float32, device=device)
-        self.rowsum = torch.empty(T, dtype=torch.int32, device=device)
-        self.glu_out = next((p.name for p in wl.projections if p.glu), None)
+            n = self.copies * wl.layers
+            self.Wp[p.name] = [Wp0] + [Wp0.clone() for _ in range(n - 1)]
+            self.beta[p.name] = [b0] + [b0.clone() for _ in range(n - 1)]
+        self.x = torch.from_numpy(synth.activations(0, "x_attn", T, H, dtype=xdt,
+                                                    outlier_frac=wl.outlier_frac,
+                                                    outlier_scale=wl.outlier_scale)).to(device)
+        self.y = [{p.name: torch.empty((T, p.N // 2 if p.glu else p.N), dtype=self.ydt,
+                                       device=device) for p in wl.projections}
+                  for _ in range(wl.layers)]
+        self.use_program = (path == "program") or (path == "auto" and T <= 64)
+        self.programs = []
+        if self.use_program:
+            for c in range(self.copies):
+                self.programs.append(mmf.Program(self.projection_list(c), T))
+        else:
+            kmax = max(p.K for p in wl.projections)
+            nmax = max(p.N for p in wl.projections)
+            self.ws = mmf.workspace(mmf.mmf_forward_workspace_bytes(T, kmax, nmax), device)
+            self.A = torch.empty((T, kmax), dtype=torch.int8, device=device)
+            self.gamma = torch.empty(T, dtype=torch.float32, device=device)
+            self.rowsum = torch.empty(T, dtype=torch.int32, device=device)
 
-    def input_of(self, p):
-        return self.y[self.glu_out] if p.src == "h" else self.x[p.src]
+    def input_of(self, l, p):
+        ys = self.y[l]
+        if p.name in ("i_proj", "f_proj", "g_proj", "proj"):
+            return self.x if l == 0 else self.y[l - 1]["down_proj"]
+        if p.name == "o_proj":
+            return ys["g_proj"]
+        if p.name == "gate_proj":
+            return ys["o_proj"]
+        return ys["gate_proj"]                      # down_proj reads the GLU output
+
+    def projection_list(self, c):
+        out = []
+        for l in range(self.wl.layers):
+            li = c * self.wl.layers + l
+            for p in self.wl.projections:
+                out.append(dict(x=self.input_of(l, p), Wp=self.Wp[p.name][li],
+                                beta=self.beta[p.name][li], y=self.y[l][p.name], glu=p.glu,
+                                level=4 * l + LEVEL_OF[p.name]))
+        return out
+
+    @property
+    def final_output(self):
+        return self.y[-1]["down_proj" if "down_proj" in self.y[-1] else "proj"]
 
     def run_step(self, step_index):
-        """One step through the public forward entry points (2 launches per projection)."""
+        """One step through the public entry points: one program launch, or two launches per
+        projection in dependency order."""
+        c = step_index % self.copies
+        if self.use_program:
+            self.programs[c].run()
+            return
         mmf = self.mmf
         for l in range(self.wl.layers):
-            li = (step_index * self.wl.layers + l) % self.n_layers_total
-            for p in self.wl.projections:
+            li = c * self.wl.layers + l
+            for p in sorted(self.wl.projections, key=lambda q: LEVEL_OF[q.name]):
                 f = mmf.mmf_bitlinear_glu_forward if p.glu else mmf.mmf_bitlinear_forward
-                f(self.input_of(p), None, 1e-8, self.Wp[p.name][li], self.beta[p.name][li],
-                  p.N, self.y[p.name], self.ws)
+                f(self.input_of(l, p), None, 1e-8, self.Wp[p.name][li], self.beta[p.name][li],
+                  p.N, self.y[l][p.name], self.ws)
 
-    def run_step_split(self, step_index, ev):
-        """The same step with the two launches of each projection bracketed by events."""
-        mmf, torch = self.mmf, self.torch
+    def run_step_timed(self, step_index, ev):
+        """The same step with every launch bracketed by CUDA events."""
+        torch, mmf = self.torch, self.mmf
+        c = step_index % self.copies
+        if self.use_program:
+            e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+            e0.record()
+            self.programs[c].run()
+            e1.record()
+            ev.append(("program", step_bytes(self.wl), self.flops_per_step, e0, e1))
+            return
         T = self.wl.T
         for l in range(self.wl.layers):
-            li = (step_index * self.wl.layers + l) % self.n_layers_total
-            for p in self.wl.projections:
+            li = c * self.wl.layers + l
+            for p in sorted(self.wl.projections, key=lambda q: LEVEL_OF[q.name]):
                 A = self.A.view(-1)[:T * p.K].view(T, p.K)
                 e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 e0.record()
-                mmf.mmf_quantize_activations(self.input_of(p), None, 1e-8, A, self.gamma,
+                mmf.mmf_quantize_activations(self.input_of(l, p), None, 1e-8, A, self.gamma,
                                              self.rowsum)
                 e1.record()
                 mmf.mmf_bitlinear_forward_quantized(A, self.gamma, self.rowsum,
                                                     self.Wp[p.name][li], self.beta[p.name][li],
-                                                    p.N, p.glu, self.y[p.name])
+                                                    p.N, p.glu, self.y[l][p.name])
                 e2.record()
-                ev.append((p, e0, e1, e2))
+                ev.append(("act_quant", quant_bytes(p, T, 4 if self.wl.x_dtype == "f32" else 2),
+                           0, e0, e1))
+                ev.append(("ternary_gemm", projection_bytes(p, T), 2 * T * p.N * p.K, e1, e2))
 
     @property
     def launches_per_step(self):
-        return 2 * len(self.wl.projections) * self.wl.layers
+        return 1 if self.use_program else 2 * len(self.wl.projections) * self.wl.layers
 
     @property
     def packed_bytes_per_step(self):
         return self.wl.packed_bytes_per_layer * self.wl.layers
+
+    @property
+    def flops_per_step(self):
+        return 2 * self.wl.T * self.wl.weights_per_layer * self.wl.layers
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -288,7 +346,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device(f"cuda:{local_rank}")
     wl = synth.WORKLOADS[args.workload]
-    g = GpuWorkload(wl, dev)
+    g = GpuWorkload(wl, dev, args.path)
     stream = torch.cuda.Stream(device=dev)
     T = wl.T
 
@@ -299,19 +357,40 @@ def run_gpu(args, rank, world, local_rank):
     if mmf.mmf_get_device_status() != 0:
         raise RuntimeError("device status reported a timeout during warm-up")
 
-    # CUDA graphs of whole steps, one per weight-copy phase
-    n_graphs = g.copies
-    graphs = []
+    # CUDA graphs: one graph runs `chunk` consecutive steps (rotating the weight copies); the
+    # timed region replays it K // chunk times plus one graph for the remaining K % chunk steps
+    chunk = g.copies if g.use_program else 1
+    chunk = max(1, min(chunk, args.steps))
+
+    def capture(n_steps):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for i in range(n_steps):
+                g.run_step(i)
+        return gr
+
     with torch.cuda.stream(stream):
-        for j in range(n_graphs):
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=stream):
-                g.run_step(j)
-            graphs.append(gr)
+        if g.use_program:
+            g_main = capture(chunk)
+            rem = args.steps % chunk
+            g_rem = capture(rem) if rem else None
+            graphs = None
+        else:
+            graphs = [capture_one(g, stream, j) for j in range(g.copies)]
     torch.cuda.synchronize()
+
+    def replay_steps(n):
+        if g.use_program:
+            for _ in range(n // chunk):
+                g_main.replay()
+            if n % chunk:
+                (g_rem if n % chunk == args.steps % chunk else capture(n % chunk)).replay()
+        else:
+            for i in range(n):
+                graphs[i % g.copies].replay()
+
     with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            graphs[i % n_graphs].replay()
+        replay_steps(max(args.warmup, 3) if not g.use_program else chunk)
     torch.cuda.synchronize()
 
     def barrier():
@@ -319,7 +398,7 @@ def run_gpu(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
-    # ---- headline: K graph replays, inputs resident in HBM
+    # ---- headline: K steps of graph replays, inputs resident in HBM
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
                       os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]) as clk:
@@ -327,8 +406,7 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             start.record()
-            for i in range(args.steps):
-                graphs[i % n_graphs].replay()
+            replay_steps(args.steps)
             end.record()
         torch.cuda.synchronize()
         barrier()
@@ -340,44 +418,54 @@ def run_gpu(args, rank, world, local_rank):
     ms_per_step = elapsed_s * 1e3 / args.steps
 
     # ---- instrumented pass: every launch bracketed by events (durations per kernel)
-    per_kernel = {"act_quant": [0.0, 0, 0.0], "ternary_gemm": [0.0, 0, 0.0]}   # ms, n, bytes
+    per_kernel = {}
     k_steps = min(args.steps, max(20, 2000 // max(1, g.launches_per_step)))
     ev = []
     with torch.cuda.stream(stream):
         torch.cuda._sleep(int(1e9))     # let the host queue the whole pass before it runs
         for i in range(k_steps):
-            g.run_step_split(i, ev)
+            g.run_step_timed(i, ev)
     torch.cuda.synchronize()
-    for p, e0, e1, e2 in ev:
-        per_kernel["act_quant"][0] += e0.elapsed_time(e1)
-        per_kernel["act_quant"][1] += 1
-        per_kernel["act_quant"][2] += quant_bytes(p, T, 4 if wl.x_dtype == "f32" else 2)
-        per_kernel["ternary_gemm"][0] += e1.elapsed_time(e2)
-        per_kernel["ternary_gemm"][1] += 1
-        per_kernel["ternary_gemm"][2] += projection_bytes(p, T)
+    for name, nbytes, nflops, e0, e1 in ev:
+        acc = per_kernel.setdefault(name, [0.0, 0, 0.0, 0.0])
+        acc[0] += e0.elapsed_time(e1)
+        acc[1] += 1
+        acc[2] += nbytes
+        acc[3] += nflops
     total_ms = sum(v[0] for v in per_kernel.values())
     kernels = {k: {"launches": v[1], "avg_us": 1e3 * v[0] / max(1, v[1]),
                    "share": v[0] / total_ms if total_ms else None,
                    "achieved_gbs": (v[2] / (v[0] / 1e3) / 1e9) if v[0] else None}
                for k, v in per_kernel.items()}
     dominant = max(per_kernel, key=lambda k: per_kernel[k][0])
-    hbm_peak, _, peak_kind = measured_peaks()
+    hbm_peak, bf16_peak, peak_kind = measured_peaks()
     dom = per_kernel[dominant]
-    achieved = dom[2] / (dom[0] / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
-                "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                "peak_source": peak_kind,
-                "bytes_per_launch": dom[2] / dom[1],
-                "traffic": profiled_traffic(dominant, wl.name)}
+    dom_s = dom[0] / 1e3
+    if T > 64 and dom[3] > 0:
+        # prefill: the contraction is bound by the int8 tensor pipe; its peak is the measured
+        # bf16 GEMM throughput times the nominal int8/bf16 ratio (2)
+        achieved = dom[3] / dom_s / 1e12
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1),
+                    "peak": round(2 * bf16_peak, 1), "unit": "TOPS",
+                    "frac": round(achieved / (2 * bf16_peak), 4),
+                    "peak_source": peak_kind + " (2 x bf16 dense, the nominal int8/bf16 ratio)",
+                    "ops_per_launch": dom[3] / dom[1], "traffic": None}
+    else:
+        achieved = dom[2] / dom_s / 1e9
+        roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
+                    "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                    "peak_source": peak_kind,
+                    "bytes_per_launch": dom[2] / dom[1],
+                    "traffic": profiled_traffic("program_kernel" if dominant == "program"
+                                                else dominant, wl.name)}
 
     # ---- e2e: the public API with host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        hx = {s: t.cpu().pin_memory() for s, t in g.x.items()}
-        outs = [p.name for p in wl.projections if not p.glu]
-        hy = {n: torch.empty_like(g.y[n], device="cpu").pin_memory() for n in outs}
-        h2d = sum(t.numel() * t.element_size() for t in hx.values())
-        d2h = sum(t.numel() * t.element_size() for t in hy.values())
+        hx = g.x.cpu().pin_memory()
+        hy = torch.empty_like(g.final_output, device="cpu").pin_memory()
+        h2d = hx.numel() * hx.element_size()
+        d2h = hy.numel() * hy.element_size()
         e2e_steps = min(args.steps, 200)
         with torch.cuda.stream(stream):
             for i in range(3):
@@ -388,61 +476,78 @@ def run_gpu(args, rank, world, local_rank):
         with torch.cuda.stream(stream):
             s0.record()
             for i in range(e2e_steps):
-                for s, t in g.x.items():
-                    t.copy_(hx[s], non_blocking=True)
+                g.x.copy_(hx, non_blocking=True)
                 g.run_step(i)
-                for n in outs:
-                    hy[n].copy_(g.y[n], non_blocking=True)
+                hy.copy_(g.final_output, non_blocking=True)
             s1.record()
         torch.cuda.synchronize()
         barrier()
         e2e_s = reduce_max(s0.elapsed_time(s1) / 1e3, world, dev)
         e2e = {"value": round(aggregate_throughput(T, e2e_steps, world, e2e_s), 1),
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "steps": e2e_steps, "path": "mmf_bitlinear_forward / _glu_forward per projection,"
-               " pinned host inputs and outputs"}
+               "steps": e2e_steps,
+               "path": ("mmf_program_run (one launch per step)" if g.use_program else
+                        "mmf_bitlinear_forward / _glu_forward per projection") +
+                       ", step input from pinned host memory, last output back to pinned host"}
 
-    for gr in graphs:
-        del gr
-    graphs.clear()
     return {
         "value": value, "ms_per_step": ms_per_step, "elapsed_s": elapsed_s, "clocks": clocks,
         "roofline": roofline, "kernels": kernels, "e2e": e2e,
         "launches": g.launches_per_step * args.steps,
         "weight_gbs": g.packed_bytes_per_step * args.steps * world / elapsed_s / 1e9,
-        "copies": g.copies,
+        "int8_tops": g.flops_per_step * args.steps * world / elapsed_s / 1e12,
+        "copies": g.copies, "path": "program" if g.use_program else "launches",
     }
+
+
+def capture_one(g, stream, j):
+    import torch
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=stream):
+        g.run_step(j)
+    return gr
 
 
 # ----------------------------------------------------------------------------- oracle arm
 def oracle_sample(wl, n_tokens):
-    """Inputs of a bounded sample of one step for the oracle: the first n_tokens tokens and
-    every projection of one layer, weights quantised by the oracle itself."""
+    """Inputs of a bounded sample of one step for the oracle: the first n_tokens tokens of the
+    step input and one layer's weights, quantised by the oracle itself."""
     import oracle
     H = wl.projections[0].K
-    xs = {s: synth.activations(0, s, wl.T, H, dtype=np.float32 if wl.x_dtype == "f32"
-                               else np.float16, outlier_frac=wl.outlier_frac,
-                               outlier_scale=wl.outlier_scale)[:n_tokens]
-          for s in {p.src for p in wl.projections if p.src != "h"}}
+    x = synth.activations(0, "x_attn", wl.T, H, dtype=np.float32 if wl.x_dtype == "f32"
+                          else np.float16, outlier_frac=wl.outlier_frac,
+                          outlier_scale=wl.outlier_scale)[:n_tokens]
     weights = {}
     for p in wl.projections:
         W = synth.weights(0, p.name, p.N, p.K)
         beta = oracle.absmean_beta(W)
         weights[p.name] = (oracle.ternary_codes(W, beta), beta)
-    return xs, weights
+    return x, weights
 
 
-def oracle_step(wl, xs, weights):
+def oracle_step(wl, x, weights):
+    """One layer of the step in the same data flow as the GPU arm (i/f/g on the input, o on
+    g's output, gate on o's output, down on the GLU output), outputs rounded to the output
+    dtype where they feed the next projection."""
     import oracle
-    h = None
-    for p in wl.projections:
-        x = h.astype(np.float16) if p.src == "h" else xs[p.src]
+    ydt = np.float32 if wl.y_dtype == "f32" else np.float16
+    outs = {}
+    for p in sorted(wl.projections, key=lambda q: LEVEL_OF[q.name]):
+        if p.name in ("i_proj", "f_proj", "g_proj", "proj"):
+            xin = x
+        elif p.name == "o_proj":
+            xin = outs["g_proj"]
+        elif p.name == "gate_proj":
+            xin = outs["o_proj"]
+        else:
+            xin = outs["gate_proj"]
         c, beta = weights[p.name]
-        q, gamma, _ = oracle.rmsnorm_actquant(x)
-        acc = oracle.ternary_accumulate(q, c)
-        y = oracle.dequant(acc, gamma, beta)
+        q, gamma, _ = oracle.rmsnorm_actquant(xin)
+        y = oracle.dequant(oracle.ternary_accumulate(q, c), gamma, beta)
         if p.glu:
-            h = oracle.silu_glu(y)
+            y = oracle.silu_glu(y)
+        outs[p.name] = y.astype(ydt)
+    return outs
 
 
 def oracle_tokens_per_s(wl, seconds, n_tokens=None):
@@ -462,7 +567,7 @@ def oracle_tokens_per_s(wl, seconds, n_tokens=None):
     tps = n_tokens * reps / el / wl.layers
     return tps, {"kind": "oracle", "cores": 1,
                  "sample": f"first {n_tokens} of {wl.T} tokens through all "
-                           f"{len(wl.projections)} projections of one layer, repeated "
+                           f"{len(wl.projections)} chained projections of one layer, repeated "
                            f"{reps} times ({el:.1f} s); tokens/s scaled by 1/{wl.layers} "
                            f"layers", "value": round(tps, 3), "unit": "tokens/s"}
 
@@ -507,6 +612,8 @@ def config_of(wl, res):
                    "activations stay L2-resident as in a layer-by-layer decode"
                    % (res["copies"], res["copies"] * wl.packed_bytes_per_layer * wl.layers / 1e6))
         c["timing"] = "CUDA graph replays of whole steps, CUDA events on the launch stream"
+        c["dataflow"] = ("per layer: i/f/g read the layer input, o reads g's output, gate reads "
+                         "o's output, down reads the GLU output, the next layer reads down's")
     return c
 
 
@@ -537,6 +644,8 @@ def main(argv=None):
                     "scaling": "weak", "vs_baseline": None, "dtype": "int8",
                     "data": "synthetic", "config": config_of(wl, res),
                     "weight_gbs": round(res["weight_gbs"], 1),
+                    "int8_tops": round(res["int8_tops"], 2),
+                    "path": res["path"],
                     "roofline": res["roofline"], "kernels": res["kernels"],
                     "clocks": res["clocks"], "e2e": res["e2e"],
                     "gpu_launches": res["launches"],

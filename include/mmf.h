@@ -137,6 +137,46 @@ mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int64_t K, con
                                       int64_t N, int32_t* acc, void* ws, size_t ws_bytes,
                                       void* stream);
 
+/* ---- a whole decode step in one launch ---------------------------------------------------- */
+
+/* One FusedBitLinear of a program.  Projections are grouped into dependency levels: the input
+ * of a level-L projection may be the output of any projection of a lower level (for example
+ * down_proj reading gate_proj's GLU output), never of the same or a higher level. */
+typedef struct {
+  const void* x;          /* input [T x K] (device), f16 or f32 */
+  mmf_dtype xdt;
+  const float* norm_w;    /* K floats or NULL (all ones) */
+  const uint8_t* Wp;      /* packed weights [N x K/4] from mmf_quantize_weights */
+  const float* beta;      /* device float */
+  int64_t K;              /* in_features: K % 128 == 0, K <= 8192 (f16) or 4096 (f32) */
+  int64_t N;              /* weight rows: N % 128 == 0 (2I for the GLU form) */
+  int32_t glu;            /* 1: SiLU-GLU epilogue, output is T x N/2 */
+  int32_t level;          /* 0-based dependency level */
+  void* y;                /* output (device), T x N (or T x N/2) */
+  mmf_dtype ydt;
+} mmf_projection;
+
+/* Workspace bytes a program of n projections at T tokens needs (plan, quantised inputs,
+ * split-K partial sums and counters).  0 if the program is not supported (T > 64, more than
+ * 1024 projections or 128 levels, or a shape outside the limits). */
+size_t mmf_program_workspace_bytes(const mmf_projection* p, int n, int64_t T);
+
+/* Plans a program into `ws` ([P1], [P3]; [P4] figure items 4 and 5, for every projection):
+ * groups projections that share an input into one quantisation, splits every level's
+ * k-blocks evenly over the SMs, encodes the tensor maps and zeroes the counters.  The
+ * pointers in `p` are baked into the plan: every later mmf_program_run reads and writes those
+ * same buffers.  Copies the plan with stream-ordered copies on `stream`.  1 <= T <= 64. */
+mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T, float eps, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Runs a planned program: one persistent launch, one CTA per SM.  Level by level, every CTA
+ * quantises a share of the level's input rows (RMSNorm + int8), then streams its share of the
+ * packed weights through the tcgen05 contraction (weights are prefetched across levels), and
+ * the level ends when every output is written.  Grid-wide waits are bounded: on a timeout the
+ * kernel records MMF_ERR_TIMEOUT (mmf_get_device_status) and returns; call mmf_program_init
+ * again before the next run in that case.  Calls on one workspace must not overlap. */
+mmf_status mmf_program_run(void* ws, void* stream);
+
 /* ---- forward without any allocation ------------------------------------------------------ */
 
 /* The pages have no counterpart to this entry point; it serves callers that cannot call

@@ -20,7 +20,8 @@ __all__ = [
     "mmf_quantize_activations", "mmf_bitlinear_forward_quantized",
     "mmf_ternary_accumulate_i32", "mmf_bitlinear_forward_noalloc", "mmf_get_device_status",
     "mmf_debug_wait_timeout_probe", "mmf_status_string", "mmf_version",
-    "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
+    "mmf_program_workspace_bytes", "mmf_program_init", "mmf_program_run", "Projection",
+    "Program", "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
     "MMF_F32", "MMF_F16", "STATUS",
 ]
 
@@ -39,6 +40,14 @@ class MMFError(RuntimeError):
     def __init__(self, fn, code):
         super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
         self.code = code
+
+
+class Projection(ctypes.Structure):
+    """Mirror of the C struct mmf_projection (one FusedBitLinear of a program)."""
+    _fields_ = [("x", ctypes.c_void_p), ("xdt", ctypes.c_int), ("norm_w", ctypes.c_void_p),
+                ("Wp", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("K", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("glu", ctypes.c_int32), ("level", ctypes.c_int32),
+                ("y", ctypes.c_void_p), ("ydt", ctypes.c_int)]
 
 
 _lib = None
@@ -64,6 +73,9 @@ def lib():
             "mmf_bitlinear_forward_quantized": ([P, P, P, I64, I64, P, P, I64, I, P, I, P], I),
             "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
             "mmf_bitlinear_forward_noalloc": ([P, I, I64, I64, P, F, P, P, I64, P, I, P], I),
+            "mmf_program_workspace_bytes": ([P, I, I64], SZ),
+            "mmf_program_init": ([P, I, I64, F, P, SZ, P], I),
+            "mmf_program_run": ([P, P], I),
             "mmf_get_device_status": ([], I),
             "mmf_debug_wait_timeout_probe": ([ctypes.c_uint64, P], I),
             "mmf_status_string": ([I], ctypes.c_char_p),
@@ -175,6 +187,49 @@ def mmf_bitlinear_forward_noalloc(x, norm_w, eps, Wp, beta, N, y, stream=None):
     _check("mmf_bitlinear_forward_noalloc", lib().mmf_bitlinear_forward_noalloc(
         _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(Wp), _ptr(beta), N, _ptr(y),
         _dt(y), _stream(stream)))
+
+
+def _proj_array(projs):
+    arr = (Projection * len(projs))()
+    for i, p in enumerate(projs):
+        x, norm_w, Wp, beta, y, glu, level = (p["x"], p.get("norm_w"), p["Wp"], p["beta"], p["y"],
+                                              p.get("glu", False), p.get("level", 0))
+        arr[i] = Projection(_ptr(x), _dt(x), _ptr(norm_w), _ptr(Wp), _ptr(beta), x.shape[1],
+                            Wp.shape[0], 1 if glu else 0, level, _ptr(y), _dt(y))
+    return arr
+
+
+def mmf_program_workspace_bytes(projs, T):
+    arr = _proj_array(projs)
+    return lib().mmf_program_workspace_bytes(arr, len(projs), T)
+
+
+def mmf_program_init(projs, T, eps, ws, stream=None):
+    arr = _proj_array(projs)
+    _check("mmf_program_init", lib().mmf_program_init(arr, len(projs), T, float(eps), _ptr(ws),
+                                                      _nbytes(ws), _stream(stream)))
+
+
+def mmf_program_run(ws, stream=None):
+    _check("mmf_program_run", lib().mmf_program_run(_ptr(ws), _stream(stream)))
+
+
+class Program:
+    """A planned list of projections run as one launch (see mmf_program_init).
+
+    ``projs`` is a list of dicts with keys x, Wp, beta, y and optionally norm_w, glu, level;
+    the tensors must stay alive and in place for as long as the program is run."""
+
+    def __init__(self, projs, T, eps=1e-8, stream=None):
+        n = mmf_program_workspace_bytes(projs, T)
+        if n == 0:
+            raise MMFError("mmf_program_workspace_bytes", 2)
+        self.projs = list(projs)
+        self.ws = workspace(n, projs[0]["x"].device)
+        mmf_program_init(self.projs, T, eps, self.ws, stream)
+
+    def run(self, stream=None):
+        mmf_program_run(self.ws, stream)
 
 
 def mmf_get_device_status():

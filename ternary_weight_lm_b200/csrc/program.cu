@@ -1,0 +1,1016 @@
+// A program of FusedBitLinear projections (a decode step) in one persistent launch.
+//
+// The projections are the ones of an HGRNBit block ("matmulfreellm 評価 ...", section "HGRNBit
+// という層構成を読む"): i/f/g/o, gate_proj with the SiLU-GLU epilogue, down_proj reading the GLU
+// output.  Each one computes what mmf_bitlinear_forward computes ("MatMul-freie LLMs: Zentrale
+// Konzepte erklärt", sections "MatMul durch ternäre Operationen ersetzen" and "Kernkomponenten:
+// MLGRU und GLU", figure items 4 and 5), with the same operation order, so the results match
+// the single-projection entry points.
+//
+// Why one launch: at decode sizes (T <= 64 tokens) a projection streams a few hundred KB to a
+// few MB of packed weights, well under a microsecond of HBM time, while every separate launch
+// costs microseconds of latency.  Here one CTA per SM runs the whole program:
+//   for each dependency level L
+//     1. the four epilogue warps of every CTA quantise a share of the level's input rows
+//        (RMSNorm + per-token absmax int8, one warp per row), then arrive on grid barrier Q[L];
+//     2. each CTA runs its planned units (a 128-row weight tile and a range of k-blocks): a
+//        TMA producer streams packed weights (ahead of time, across levels: weights do not
+//        depend on activations) and, once Q[L] has passed, the activation codes; four warps
+//        unpack the 2-bit codes into TMEM; one thread issues tcgen05 kind::i8 MMAs into one of
+//        two TMEM accumulators; the epilogue dequantises (and applies the GLU) or, for a tile
+//        split over several CTAs, hands its int32 partial sum to whichever CTA finishes the
+//        tile last, which adds the partials in split order (exact) and finalises the tile;
+//     3. every CTA arrives on grid barrier O[L]; the next level may read this level's outputs.
+// Grid barriers are counters in the workspace with bounded waits; a timeout anywhere sets a
+// poison flag that makes every other wait give up too, and is reported as MMF_ERR_TIMEOUT.
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/mmf.h"
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+#define MMF_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace mmf {
+namespace {
+
+constexpr int kPThreads = 192;
+constexpr int kPEpi = 128;
+constexpr int kPKB = 128;                  // K per stage
+constexpr int kPWRow = kPKB / 4;           // packed bytes per weight row per stage
+constexpr int kPWStage = 128 * kPWRow;     // 4 KB
+constexpr int kPStages = 12;               // SMEM stages == TMEM slots
+constexpr int kPACol0 = 128;               // TMEM: accumulators at 0 and 64, slots from 128
+constexpr int kMaxLevels = 128;
+constexpr int kMaxProj = 1024;
+constexpr int kMaxSplit = 16;
+constexpr int kMinSplitKb = 8;             // latency beats spreading at decode sizes
+constexpr uint64_t kPDrainNs = 2000000000ull;
+
+struct PProj {
+  const uint8_t* Wp;
+  const float* beta;
+  void* y;
+  int32_t K, N, glu, ydt, in, level, wmap, pad;
+};
+
+struct PIn {
+  const void* x;
+  const float* g;
+  int8_t* A;
+  float* gamma;
+  int32_t* rowsum;
+  int32_t K, xdt, level, amap;
+};
+
+struct PUnit {
+  int32_t proj, tile, kb0, nkb, split, nsplit, tile_id, part_off;
+};
+
+struct PHeader {
+  int32_t n_proj, n_in, n_levels, n_ctas, n_units, T, BN, n_tiles;
+  float eps;
+  int32_t pad[3];
+  int64_t off_in, off_proj, off_units, off_ctaoff, off_maps, off_tilectr, off_levelctr, off_part;
+  int32_t in_begin[kMaxLevels + 1];
+};
+
+template <int BN>
+struct PCfg {
+  static constexpr int kAct = BN * kPKB;
+  static constexpr int kStage = kAct + kPWStage;
+  static constexpr int kBar = (8 * (3 * kPStages + 5) + 127) / 128 * 128;   // keeps what follows 128-byte aligned
+  static constexpr int kXbuf = BN * 64 * 4;      // GLU exchange: multiplier half, fp32
+  static constexpr int kTok = 8 * 64;            // per-token scale and code sum
+  static constexpr int kOst = BN * 128 * 2;      // fp16 output staging [token][column]
+  static constexpr int kSmem = 1024 + kPStages * kStage + kBar + kXbuf + kTok + kOst + 64;
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kSmem >= 118 * 1024 || BN < 64, "one CTA per SM");
+};
+
+// ------------------------------------------------------------------------------ device helpers
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Arrive on a grid barrier: one fire-and-forget reduction with release semantics (orders this
+// thread's earlier writes, and those of the CTA published to it by a preceding bar.sync).
+__device__ __forceinline__ void grid_arrive(unsigned* ctr) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
+// Waits until *ctr >= target.  Bounded: gives up after limit_ns, or at once when the poison
+// flag is set (another CTA timed out); a timeout sets the poison flag and the status word.
+__device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, unsigned* poison,
+                                          uint64_t limit_ns, unsigned* status) {
+  if (ld_acquire_u32(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire_u32(ctr) >= target) return true;
+    if (ld_acquire_u32(poison) != 0u) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicExch(poison, 1u);
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void widen16(const uint4& a, int xdt, float (&v)[8], int& n) {
+  if (xdt == kInF16) {
+    const __half2* h = reinterpret_cast<const __half2*>(&a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+    n = 8;
+  } else {
+    v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+    v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+    n = 4;
+  }
+}
+
+// The 128 epilogue threads quantise row t of input `in` together: the same operations, in the
+// same order, as the activation pre-pass kernel (mean of squares in double, rounded once;
+// inv = 1/sqrt(ms+eps); xhat = (x*inv)*g; gamma = max|xhat| floored at 1e-5;
+// q = rne(xhat * (127/gamma))).  The row is read once (ld.global.cg: this launch may have
+// written it) into registers, at most 8 vectors of 16 bytes per thread (K <= 8192 fp16 /
+// 4096 fp32).  red_d/red_f/red_i: per-warp partials in shared memory.
+__device__ void quant_row(const PIn in, int t, float eps, int et, double* red_d, float* red_f,
+                          int* red_i) {
+  constexpr int kVmax = 8;
+  const int K = in.K;
+  const int E = in.xdt == kInF16 ? 8 : 4;
+  const int nvec = K / E;
+  const int lane = et & 31, w = et >> 5;
+  const uint4* xr = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(in.x) +
+                                                   static_cast<int64_t>(t) * K * (E == 8 ? 2 : 4));
+  uint4 raw[kVmax];
+#pragma unroll
+  for (int i = 0; i < kVmax; ++i) {
+    const int vi = et + kPEpi * i;
+    if (vi < nvec) raw[i] = __ldcg(xr + vi);
+  }
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < kVmax; ++i) {
+    if (et + kPEpi * i < nvec) {
+      float v[8];
+      int n;
+      widen16(raw[i], in.xdt, v, n);
+      for (int e = 0; e < n; ++e) {
+        const double d = static_cast<double>(v[e]);
+        ss = __fma_rn(d, d, ss);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red_d[w] = ss;
+  named_bar_sync(1, kPEpi);
+  ss = red_d[0] + red_d[1] + red_d[2] + red_d[3];
+  const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
+  const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kVmax; ++i) {
+    const int vi = et + kPEpi * i;
+    if (vi < nvec) {
+      float v[8];
+      int n;
+      widen16(raw[i], in.xdt, v, n);
+      for (int e = 0; e < n; ++e) {
+        const float gk = in.g ? __ldg(in.g + vi * E + e) : 1.0f;
+        amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), gk)));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) red_f[w] = amax;
+  named_bar_sync(1, kPEpi);
+  amax = fmaxf(fmaxf(red_f[0], red_f[1]), fmaxf(red_f[2], red_f[3]));
+  const float gm = fmaxf(amax, 1e-5f);
+  const float s = __fdiv_rn(127.0f, gm);
+  int rs = 0;
+  int8_t* ar = in.A + static_cast<int64_t>(t) * K;
+#pragma unroll
+  for (int i = 0; i < kVmax; ++i) {
+    const int vi = et + kPEpi * i;
+    if (vi < nvec) {
+      float v[8];
+      int n;
+      widen16(raw[i], in.xdt, v, n);
+      uint32_t wd[2] = {0u, 0u};
+      for (int e = 0; e < n; ++e) {
+        const float gk = in.g ? __ldg(in.g + vi * E + e) : 1.0f;
+        const float xh = __fmul_rn(__fmul_rn(v[e], inv_r), gk);
+        int q = __float2int_rn(__fmul_rn(xh, s));
+        q = max(-128, min(127, q));
+        rs += q;
+        wd[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (e & 3));
+      }
+      if (E == 8)
+        *reinterpret_cast<uint2*>(ar + vi * 8) = make_uint2(wd[0], wd[1]);
+      else
+        *reinterpret_cast<uint32_t*>(ar + vi * 4) = wd[0];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+  if (lane == 0) red_i[w] = rs;
+  named_bar_sync(1, kPEpi);
+  if (et == 0) {
+    in.gamma[t] = gm;
+    in.rowsum[t] = red_i[0] + red_i[1] + red_i[2] + red_i[3];
+  }
+  named_bar_sync(1, kPEpi);   // the scratch is reused by the next row
+}
+
+__device__ __forceinline__ void unpack_word4(uint32_t w, uint32_t* out) {
+  out[0] = w & 0x03030303u;
+  out[1] = (w >> 2) & 0x03030303u;
+  out[2] = (w >> 4) & 0x03030303u;
+  out[3] = (w >> 6) & 0x03030303u;
+}
+
+// Dequantise (and GLU) one finished tile held as int32 sums acc[j] (token j, tile row r).
+// tsc/trs: per-token scale (gamma/127 * beta) and code sum, staged in shared memory.
+// fp16 outputs go through ostage ([token][column] fp16) so that each token's 128 (or 64 GLU)
+// outputs leave as 16-byte stores; fp32 outputs are stored directly.
+template <int BN>
+__device__ __forceinline__ void finalize_tile(const PProj pj, int tile, int T,
+                                              const int32_t (&acc)[BN], int r,
+                                              const float* __restrict__ tsc,
+                                              const int32_t* __restrict__ trs,
+                                              float* __restrict__ xbuf,
+                                              __half* __restrict__ ostage) {
+  const int et = threadIdx.x - 64;
+  // pass 1 (loads and arithmetic only, so the 64 independent tokens overlap): dequantised
+  // values of this thread's row in registers
+  float v[BN];
+#pragma unroll
+  for (int j = 0; j < BN; ++j) v[j] = j < T ? static_cast<float>(acc[j] - trs[j]) * tsc[j] : 0.0f;
+  if (!pj.glu) {
+    if (pj.ydt == MMF_F16) {
+#pragma unroll
+      for (int j = 0; j < BN; ++j)
+        if (j < T) ostage[j * 128 + r] = __float2half_rn(v[j]);
+      named_bar_sync(1, kPEpi);
+      // T rows of 128 fp16 = 16 chunks of 16 bytes per row
+      for (int c = et; c < T * 16; c += kPEpi) {
+        const int j = c >> 4, k8 = (c & 15) * 8;
+        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(pj.y) + static_cast<int64_t>(j) * pj.N +
+                                  static_cast<int64_t>(tile) * 128 + k8) =
+            *reinterpret_cast<const uint4*>(ostage + j * 128 + k8);
+      }
+    } else {
+      const int64_t n = static_cast<int64_t>(tile) * 128 + r;
+#pragma unroll
+      for (int j = 0; j < BN; ++j)
+        if (j < T) reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * pj.N + n] = v[j];
+    }
+  } else {
+    // rows 0-63 of the tile are the gated half, rows 64-127 the multiplier half
+    if (r >= 64) {
+#pragma unroll
+      for (int j = 0; j < BN; ++j)
+        if (j < T) xbuf[j * 64 + (r - 64)] = v[j];
+    }
+    named_bar_sync(1, kPEpi);
+    const int64_t I = pj.N / 2;
+    if (r < 64) {
+      float u[BN];
+#pragma unroll
+      for (int j = 0; j < BN; ++j) u[j] = j < T ? xbuf[j * 64 + r] : 0.0f;
+#pragma unroll
+      for (int j = 0; j < BN; ++j) v[j] = __fdividef(v[j], 1.0f + expf(-v[j])) * u[j];
+      if (pj.ydt == MMF_F16) {
+#pragma unroll
+        for (int j = 0; j < BN; ++j)
+          if (j < T) ostage[j * 64 + r] = __float2half_rn(v[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < BN; ++j)
+          if (j < T)
+            reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * I + static_cast<int64_t>(tile) * 64 + r] = v[j];
+      }
+    }
+    named_bar_sync(1, kPEpi);
+    if (pj.ydt == MMF_F16) {
+      // T rows of 64 fp16 = 8 chunks of 16 bytes per row
+      for (int c = et; c < T * 8; c += kPEpi) {
+        const int j = c >> 3, k8 = (c & 7) * 8;
+        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(pj.y) + static_cast<int64_t>(j) * I +
+                                  static_cast<int64_t>(tile) * 64 + k8) =
+            *reinterpret_cast<const uint4*>(ostage + j * 64 + k8);
+      }
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kPThreads, 1)
+program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_ns) {
+  using C = PCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* s_act = smem;
+  uint8_t* s_w = smem + kPStages * C::kAct;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + kPStages * kPWStage);
+  float* xbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::kBar);
+  float* tsc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(xbuf) + C::kXbuf);
+  int32_t* trs = reinterpret_cast<int32_t*>(tsc + 64);
+  __half* ostage = reinterpret_cast<__half*>(trs + 64);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_flag;
+  __shared__ int s_qflag;
+  __shared__ double s_red_d[4];
+  __shared__ float s_red_f[4];
+  __shared__ int s_red_i[4];
+
+  auto full = [&](int s) { return smem_u32(bars + s); };
+  auto afull = [&](int s) { return smem_u32(bars + kPStages + s); };
+  auto empty = [&](int s) { return smem_u32(bars + 2 * kPStages + s); };
+  auto accfull = [&](int b) { return smem_u32(bars + 3 * kPStages + b); };
+  auto accempty = [&](int b) { return smem_u32(bars + 3 * kPStages + 2 + b); };
+  const uint32_t drainbar = smem_u32(bars + 3 * kPStages + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(afull(s), 4);
+      mbar_init(empty(s), 1 + 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull(b), 1);
+      mbar_init(accempty(b), 4);
+    }
+    mbar_init(drainbar, 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  pdl_wait();
+  // the plan in the workspace is read only after the wait
+  const PHeader& H = *reinterpret_cast<const PHeader*>(ws);
+  const PIn* ins = reinterpret_cast<const PIn*>(ws + H.off_in);
+  const PProj* projs = reinterpret_cast<const PProj*>(ws + H.off_proj);
+  const PUnit* units = reinterpret_cast<const PUnit*>(ws + H.off_units);
+  const int32_t* ctaoff = reinterpret_cast<const int32_t*>(ws + H.off_ctaoff);
+  const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(ws + H.off_maps);
+  unsigned* tilectr = reinterpret_cast<unsigned*>(const_cast<uint8_t*>(ws) + H.off_tilectr);
+  unsigned* lvl = reinterpret_cast<unsigned*>(const_cast<uint8_t*>(ws) + H.off_levelctr);
+  unsigned* poison = lvl + 2 * kMaxLevels;
+  unsigned* exitctr = lvl + 2 * kMaxLevels + 1;
+  int32_t* parts = reinterpret_cast<int32_t*>(const_cast<uint8_t*>(ws) + H.off_part);
+
+  const int nct = H.n_ctas;
+  const int u_begin = ctaoff[blockIdx.x], u_end = ctaoff[blockIdx.x + 1];
+  const int T = H.T;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_a = l2_policy_evict_last();
+      // The unit records are read from the workspace once per unit into registers (the TMA
+      // asm statements clobber memory, so a record read inside the stage loop would be
+      // re-fetched from L2 for every stage).
+      struct Cur {
+        int ui, k, nkb, kb0, r0, r1, level;
+        const CUtensorMap* wmap;
+        const CUtensorMap* amap;
+      };
+      auto load_cur = [&](Cur& c, int ui) {
+        c.ui = ui;
+        c.k = 0;
+        if (ui >= u_end) return;
+        const PUnit u = units[ui];
+        const PProj pj = projs[u.proj];
+        c.nkb = u.nkb;
+        c.kb0 = u.kb0;
+        c.level = pj.level;
+        if (pj.glu) {
+          c.r0 = u.tile * 64;
+          c.r1 = pj.N / 2 + u.tile * 64;
+        } else {
+          c.r0 = u.tile * 128;
+          c.r1 = c.r0 + 64;
+        }
+        c.wmap = maps + pj.wmap;
+        c.amap = maps + ins[pj.in].amap;
+      };
+      Cur wc, ac;
+      load_cur(wc, u_begin);
+      ac = wc;
+      int64_t wi = 0, ai = 0;
+      int q_level = -1;
+      bool ok = true;
+      while (ok && ac.ui < u_end) {
+        // 1. the activation tile of every stage whose weights are already requested (the
+        //    weights ran ahead); at a new level, first wait until its codes exist
+        while (ai < wi) {
+          if (ac.level > q_level) {
+            if (!grid_wait(lvl + 2 * ac.level, static_cast<unsigned>(nct), poison, limit_ns,
+                           status)) {
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            q_level = ac.level;
+          }
+          const int s = static_cast<int>(ai % kPStages);
+          tma_load_2d(smem_u32(s_act + s * C::kAct), ac.amap, full(s), (ac.kb0 + ac.k) * kPKB, 0,
+                      pol_a);
+          ++ai;
+          if (++ac.k == ac.nkb) load_cur(ac, ac.ui + 1);
+        }
+        if (!ok || wc.ui >= u_end) continue;
+        // 2. the packed weights of the next stage, up to a full ring ahead (they do not depend
+        //    on any activation)
+        const int s = static_cast<int>(wi % kPStages);
+        if (wi >= kPStages &&
+            !mbar_wait_bounded(empty(s), static_cast<uint32_t>(((wi / kPStages) - 1) & 1),
+                               limit_ns, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        const int kg = wc.kb0 + wc.k;
+        mbar_arrive_expect_tx(full(s), C::kStage);
+        uint8_t* wdst = s_w + s * kPWStage;
+        tma_load_2d(smem_u32(wdst), wc.wmap, full(s), kg * kPWRow, wc.r0, pol_w);
+        tma_load_2d(smem_u32(wdst + kPWStage / 2), wc.wmap, full(s), kg * kPWRow, wc.r1, pol_w);
+        ++wi;
+        if (++wc.k == wc.nkb) load_cur(wc, wc.ui + 1);
+      }
+      // Abort path: stages whose weights were requested but whose activation tile was not
+      // get it now (the workspace buffer is valid memory), so that every started stage
+      // completes; then wait until every copy this thread started has landed.
+      while (ai < wi && ac.ui < u_end) {
+        const int s = static_cast<int>(ai % kPStages);
+        tma_load_2d(smem_u32(s_act + s * C::kAct), ac.amap, full(s), (ac.kb0 + ac.k) * kPKB, 0,
+                    pol_a);
+        ++ai;
+        if (++ac.k == ac.nkb) load_cur(ac, ac.ui + 1);
+      }
+      for (int64_t i = wi > kPStages ? wi - kPStages : 0; i < wi; ++i)
+        mbar_wait_bounded(full(static_cast<int>(i % kPStages)),
+                          static_cast<uint32_t>((i / kPStages) & 1), kPDrainNs, nullptr, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
+      const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      int n = 0;
+      int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
+      for (int ui = u_begin; ui < u_end && ok; ++ui, ++n) {
+        const int nkb = next_nkb;
+        if (ui + 1 < u_end) next_nkb = units[ui + 1].nkb;   // overlaps this unit's MMAs
+        const int b = n & 1;
+        if (n >= 2 &&
+            !mbar_wait_bounded(accempty(b), static_cast<uint32_t>(((n >> 1) - 1) & 1), limit_ns,
+                               abort_flag, status))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(b * 64);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_bounded(afull(s), ph, limit_ns, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kAct) >> 4);
+          const uint32_t ad = tmem + kPACol0 + s * 32;
+          tc_mma_i8_ts(d, ad, bd, idesc, kb > 0 ? 1u : 0u);
+          tc_mma_i8_ts(d, ad + 8, bd + 2, idesc, 1u);
+          tc_mma_i8_ts(d, ad + 16, bd + 4, idesc, 1u);
+          tc_mma_i8_ts(d, ad + 24, bd + 6, idesc, 1u);
+          tc_commit(empty(s));
+          if (++s == kPStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (ok) tc_commit(accfull(b));
+      }
+      // Drain: nothing this thread issued may still be running when TMEM is freed.
+      tc_commit(drainbar);
+      mbar_wait_bounded(drainbar, 0u, kPDrainNs, nullptr, status);
+    }
+  } else {
+    // ------------------------------------------------------------------ quantise, unpack, epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    bool ok = true;
+    int s = 0;
+    uint32_t ph = 0;
+    int n = 0;
+    int ui = u_begin;
+    for (int L = 0; L < H.n_levels; ++L) {
+      // 1. quantise a share of this level's input rows (one warp per row)
+      const int ib = H.in_begin[L], ie = H.in_begin[L + 1];
+      const int rows = (ie - ib) * T;
+      for (int rho = blockIdx.x; rho < rows && ok; rho += nct)
+        quant_row(ins[ib + rho / T], rho % T, H.eps, et, s_red_d, s_red_f, s_red_i);
+      fence_proxy_async_global();   // the codes are read by TMA (async proxy) in other CTAs
+      named_bar_sync(1, kPEpi);
+      if (et == 0) {
+        grid_arrive(lvl + 2 * L);
+        // gamma and the code sums of this level are read below (staged per unit): wait until
+        // every CTA has quantised its rows (the unpack would wait for this anyway, through the
+        // activation tiles the producer loads after the same barrier)
+        s_qflag = grid_wait(lvl + 2 * L, static_cast<unsigned>(nct), poison, limit_ns, status) ? 1 : 0;
+        if (!s_qflag) *abort_flag = 1;
+      }
+      named_bar_sync(1, kPEpi);
+      if (!s_qflag) ok = false;
+      // 2. this CTA's units of level L
+      while (ui < u_end && projs[units[ui].proj].level == L) {
+        // plan records are copied into registers (output stores cannot alias them) and the
+        // per-token scale and code sum are staged before the unpack, so their L2 latency
+        // overlaps it
+        const PUnit u = units[ui];
+        const PProj pj = projs[u.proj];
+        const PIn in = ins[pj.in];
+        if (et < T) {
+          tsc[et] = __fmul_rn(__fdiv_rn(__ldcg(in.gamma + et), 127.0f), __ldg(pj.beta));
+          trs[et] = __ldcg(in.rowsum + et);
+        }
+        for (int kb = 0; kb < u.nkb && ok; ++kb) {
+          const bool w = mbar_wait_bounded(full(s), ph, limit_ns, abort_flag, status);
+          if (!__all_sync(0xFFFFFFFFu, w)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* wrow = s_w + s * kPWStage + r * kPWRow;
+          const int sw = (r >> 2) & 1;
+          const uint4 lo = *reinterpret_cast<const uint4*>(wrow + 16 * sw);
+          const uint4 hi = *reinterpret_cast<const uint4*>(wrow + 16 * (sw ^ 1));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty(s));
+          uint32_t uu[32];
+          unpack_word4(lo.x, uu + 0);
+          unpack_word4(lo.y, uu + 4);
+          unpack_word4(lo.z, uu + 8);
+          unpack_word4(lo.w, uu + 12);
+          unpack_word4(hi.x, uu + 16);
+          unpack_word4(hi.y, uu + 20);
+          unpack_word4(hi.z, uu + 24);
+          unpack_word4(hi.w, uu + 28);
+          tc_st_32x32b_x32(tmem + lane_addr + kPACol0 + s * 32, uu);
+          tc_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(afull(s));
+          if (++s == kPStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        // epilogue of unit ui
+        const int b = n & 1;
+        if (ok) {
+          const bool w = mbar_wait_bounded(accfull(b), static_cast<uint32_t>((n >> 1) & 1),
+                                           limit_ns, abort_flag, status);
+          ok = __all_sync(0xFFFFFFFFu, w);
+        }
+        ok = named_bar_and(1, kPEpi, ok);
+        if (!ok) break;
+        tc_fence_after();
+        int32_t acc[BN];
+        {
+          uint32_t v[32];
+#pragma unroll
+          for (int c0 = 0; c0 < BN; c0 += (BN < 32 ? BN : 32)) {
+            if constexpr (BN < 32) {
+              tc_ld_32x32b_x16(tmem + lane_addr + static_cast<uint32_t>(b * 64 + c0), v);
+            } else {
+              tc_ld_32x32b_x32(tmem + lane_addr + static_cast<uint32_t>(b * 64 + c0), v);
+            }
+            tc_wait_ld();
+#pragma unroll
+            for (int j = 0; j < (BN < 32 ? BN : 32); ++j) acc[c0 + j] = static_cast<int32_t>(v[j]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(accempty(b));
+        named_bar_sync(1, kPEpi);   // tsc/trs written by other threads
+        if (u.nsplit == 1) {
+          finalize_tile<BN>(pj, u.tile, T, acc, r, tsc, trs, xbuf, ostage);
+        } else {
+          int32_t* mine = parts + static_cast<int64_t>(u.part_off + u.split) * BN * 128;
+#pragma unroll
+          for (int j = 0; j < BN; ++j) __stcg(mine + j * 128 + r, acc[j]);
+          __threadfence();
+          named_bar_sync(1, kPEpi);
+          if (et == 0) s_flag = (atomicAdd(tilectr + u.tile_id, 1u) == static_cast<unsigned>(u.nsplit - 1));
+          named_bar_sync(1, kPEpi);
+          if (s_flag) {
+            __threadfence();
+            // add the other splits in split order (int32: exact in any order)
+            for (int sp = 0; sp < u.nsplit; ++sp) {
+              if (sp == u.split) continue;
+              const int32_t* other = parts + static_cast<int64_t>(u.part_off + sp) * BN * 128;
+#pragma unroll
+              for (int j = 0; j < BN; ++j) acc[j] += __ldcg(other + j * 128 + r);
+            }
+            finalize_tile<BN>(pj, u.tile, T, acc, r, tsc, trs, xbuf, ostage);
+            if (et == 0) tilectr[u.tile_id] = 0u;   // ready for the next run
+          }
+          named_bar_sync(1, kPEpi);
+        }
+        named_bar_sync(1, kPEpi);
+        ++n;
+        ++ui;
+      }
+      // 3. this level's outputs are written once every CTA arrives
+      named_bar_sync(1, kPEpi);
+      if (et == 0) {
+        grid_arrive(lvl + 2 * L + 1);
+        s_flag = grid_wait(lvl + 2 * L + 1, static_cast<unsigned>(nct), poison, limit_ns, status) ? 1 : 0;
+        if (!s_flag) *abort_flag = 1;
+      }
+      named_bar_sync(1, kPEpi);
+      if (!s_flag || !ok) {
+        ok = false;
+        // keep arriving on the remaining levels so that no other CTA waits for this one
+        for (int L2 = L + 1; L2 < H.n_levels; ++L2)
+          if (et == 0) {
+            grid_arrive(lvl + 2 * L2);
+            grid_arrive(lvl + 2 * L2 + 1);
+          }
+        break;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(exitctr, 1u) == static_cast<unsigned>(nct - 1)) {
+      // last CTA out: every other CTA is done with the counters, reset them for the next run
+      // (the poison flag stays set after a timeout until the program is planned again)
+      for (int L = 0; L < H.n_levels; ++L) {
+        lvl[2 * L] = 0u;
+        lvl[2 * L + 1] = 0u;
+      }
+      *exitctr = 0u;
+      __threadfence();
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ host planning
+struct Plan {
+  std::vector<PIn> ins;
+  std::vector<PProj> projs;
+  std::vector<PUnit> units;
+  std::vector<int32_t> ctaoff;
+  PHeader h;
+  size_t bytes = 0;
+  std::vector<CUtensorMap> maps;
+  std::vector<std::pair<size_t, size_t>> in_buf;   // offset of A, and of gamma/rowsum, per input
+  int BN = 0;
+};
+
+size_t al(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+mmf_status validate(const mmf_projection* p, int n, int64_t T) {
+  if (!p || n < 1 || n > kMaxProj) return MMF_ERR_INVALID_ARG;
+  if (T < 1 || T > 64) return MMF_ERR_UNSUPPORTED_SHAPE;
+  for (int i = 0; i < n; ++i) {
+    const mmf_projection& q = p[i];
+    if (!q.x || !q.Wp || !q.beta || !q.y) return MMF_ERR_INVALID_ARG;
+    if ((q.xdt != MMF_F16 && q.xdt != MMF_F32) || (q.ydt != MMF_F16 && q.ydt != MMF_F32))
+      return MMF_ERR_INVALID_ARG;
+    if (q.glu != 0 && q.glu != 1) return MMF_ERR_INVALID_ARG;
+    if (q.level < 0 || q.level >= kMaxLevels) return MMF_ERR_INVALID_ARG;
+    const int64_t kmax = q.xdt == MMF_F16 ? 8192 : 4096;
+    if (q.K < 128 || q.K > kmax || q.K % 128 != 0) return MMF_ERR_UNSUPPORTED_SHAPE;
+    if (q.N < 128 || q.N > (1 << 20) || q.N % 128 != 0) return MMF_ERR_UNSUPPORTED_SHAPE;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(q.x) | reinterpret_cast<uintptr_t>(q.Wp) |
+                        reinterpret_cast<uintptr_t>(q.y) |
+                        reinterpret_cast<uintptr_t>(q.norm_w ? q.norm_w : q.x);
+    if ((a & 15u) != 0 || (reinterpret_cast<uintptr_t>(q.beta) & 3u) != 0) return MMF_ERR_ALIGNMENT;
+  }
+  return MMF_OK;
+}
+
+// Builds the plan (without device addresses of the workspace regions, which `base` supplies).
+mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uintptr_t base,
+                      int nct, Plan& P) {
+  mmf_status st = validate(p, n, T);
+  if (st != MMF_OK) return st;
+  P = Plan();
+  P.BN = T <= 16 ? 16 : (T <= 32 ? 32 : 64);
+  int n_levels = 0;
+  for (int i = 0; i < n; ++i) n_levels = std::max(n_levels, p[i].level + 1);
+  // inputs: one per distinct (x, norm_w, K, dtype, level), ordered by level
+  std::vector<int> order(n);
+  for (int i = 0; i < n; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return p[a].level < p[b].level; });
+  std::vector<int> proj_in(n, -1);
+  for (int oi = 0; oi < n; ++oi) {
+    const int i = order[oi];
+    int found = -1;
+    for (size_t k = 0; k < P.ins.size(); ++k) {
+      const PIn& in = P.ins[k];
+      if (in.x == p[i].x && in.g == p[i].norm_w && in.K == p[i].K && in.level == p[i].level &&
+          in.xdt == (p[i].xdt == MMF_F16 ? kInF16 : kInF32)) {
+        found = static_cast<int>(k);
+        break;
+      }
+    }
+    if (found < 0) {
+      PIn in = {};
+      in.x = p[i].x;
+      in.g = p[i].norm_w;
+      in.K = static_cast<int32_t>(p[i].K);
+      in.xdt = p[i].xdt == MMF_F16 ? kInF16 : kInF32;
+      in.level = p[i].level;
+      found = static_cast<int>(P.ins.size());
+      P.ins.push_back(in);
+    }
+    proj_in[i] = found;
+  }
+  // projections: kept in caller order, weight map index = projection index
+  int tiles = 0;
+  std::vector<int> tile_base(n);
+  for (int i = 0; i < n; ++i) {
+    PProj q = {};
+    q.Wp = p[i].Wp;
+    q.beta = p[i].beta;
+    q.y = p[i].y;
+    q.K = static_cast<int32_t>(p[i].K);
+    q.N = static_cast<int32_t>(p[i].N);
+    q.glu = p[i].glu;
+    q.ydt = p[i].ydt;
+    q.in = proj_in[i];
+    q.level = p[i].level;
+    q.wmap = i;
+    P.projs.push_back(q);
+    tile_base[i] = tiles;
+    tiles += static_cast<int>(p[i].N / 128);
+  }
+  // units: per level, split every tile's k-blocks so the level's work spreads over all SMs,
+  // then assign longest-first to the least loaded CTA
+  std::vector<std::vector<PUnit>> per_cta(nct);
+  int part_slots = 0;
+  for (int L = 0; L < n_levels; ++L) {
+    int64_t work = 0;
+    for (int i = 0; i < n; ++i)
+      if (p[i].level == L) work += (p[i].N / 128) * (p[i].K / kPKB);
+    if (work == 0) continue;
+    const int64_t target = std::max<int64_t>(kMinSplitKb, (work + nct - 1) / nct);
+    std::vector<PUnit> lu;
+    for (int i = 0; i < n; ++i) {
+      if (p[i].level != L) continue;
+      const int nkb = static_cast<int>(p[i].K / kPKB);
+      const int ns = static_cast<int>(std::min<int64_t>(
+          {static_cast<int64_t>(kMaxSplit), static_cast<int64_t>(nkb), (nkb + target - 1) / target}));
+      for (int t = 0; t < p[i].N / 128; ++t) {
+        const int part_off = ns > 1 ? part_slots : 0;
+        if (ns > 1) part_slots += ns;
+        for (int sp = 0; sp < ns; ++sp) {
+          PUnit u;
+          u.proj = i;
+          u.tile = t;
+          u.kb0 = sp * nkb / ns;
+          u.nkb = (sp + 1) * nkb / ns - u.kb0;
+          u.split = sp;
+          u.nsplit = ns;
+          u.tile_id = tile_base[i] + t;
+          u.part_off = part_off;
+          lu.push_back(u);
+        }
+      }
+    }
+    std::stable_sort(lu.begin(), lu.end(), [](const PUnit& a, const PUnit& b) { return a.nkb > b.nkb; });
+    std::vector<int64_t> load(nct, 0);
+    for (const PUnit& u : lu) {
+      const int c = static_cast<int>(std::min_element(load.begin(), load.end()) - load.begin());
+      load[c] += u.nkb + 2;   // +2: per-unit set-up and epilogue cost, in k-block units
+      per_cta[c].push_back(u);
+    }
+  }
+  P.ctaoff.push_back(0);
+  for (int c = 0; c < nct; ++c) {
+    for (const PUnit& u : per_cta[c]) P.units.push_back(u);
+    P.ctaoff.push_back(static_cast<int32_t>(P.units.size()));
+  }
+  // workspace layout
+  PHeader& h = P.h;
+  std::memset(&h, 0, sizeof(h));
+  h.n_proj = n;
+  h.n_in = static_cast<int32_t>(P.ins.size());
+  h.n_levels = n_levels;
+  h.n_ctas = nct;
+  h.n_units = static_cast<int32_t>(P.units.size());
+  h.T = static_cast<int32_t>(T);
+  h.BN = P.BN;
+  h.n_tiles = tiles;
+  h.eps = eps;
+  size_t off = al(sizeof(PHeader), 256);
+  h.off_in = static_cast<int64_t>(off);
+  off = al(off + P.ins.size() * sizeof(PIn), 256);
+  h.off_proj = static_cast<int64_t>(off);
+  off = al(off + P.projs.size() * sizeof(PProj), 256);
+  h.off_units = static_cast<int64_t>(off);
+  off = al(off + P.units.size() * sizeof(PUnit), 256);
+  h.off_ctaoff = static_cast<int64_t>(off);
+  off = al(off + P.ctaoff.size() * sizeof(int32_t), 256);
+  h.off_maps = static_cast<int64_t>(off);
+  off = al(off + (P.projs.size() + P.ins.size()) * sizeof(CUtensorMap), 256);
+  h.off_tilectr = static_cast<int64_t>(off);
+  off = al(off + static_cast<size_t>(tiles) * 4, 256);
+  h.off_levelctr = static_cast<int64_t>(off);
+  off = al(off + (2 * kMaxLevels + 2) * 4, 256);
+  for (size_t k = 0; k < P.ins.size(); ++k) {
+    const size_t a_off = off;
+    off = al(off + static_cast<size_t>(T) * P.ins[k].K, 256);
+    const size_t v_off = off;
+    off = al(off + static_cast<size_t>(T) * 8, 256);
+    P.in_buf.push_back({a_off, v_off});
+    P.ins[k].A = reinterpret_cast<int8_t*>(base + a_off);
+    P.ins[k].gamma = reinterpret_cast<float*>(base + v_off);
+    P.ins[k].rowsum = reinterpret_cast<int32_t*>(base + v_off + static_cast<size_t>(T) * 4);
+    P.ins[k].amap = n + static_cast<int32_t>(k);
+  }
+  h.off_part = static_cast<int64_t>(off);
+  off = al(off + static_cast<size_t>(part_slots) * P.BN * 128 * 4, 256);
+  P.bytes = off;
+  int k = 0;
+  for (int L = 0; L <= n_levels; ++L) {
+    while (k < static_cast<int>(P.ins.size()) && P.ins[k].level < L) ++k;
+    h.in_begin[L] = k;
+  }
+  h.in_begin[n_levels] = static_cast<int32_t>(P.ins.size());
+  return MMF_OK;
+}
+
+struct RunInfo {
+  int BN;
+  int nct;
+};
+std::mutex g_runs_mu;
+std::unordered_map<const void*, RunInfo> g_runs;
+
+template <int BN>
+cudaError_t launch_program(const void* ws, int nct, unsigned* status, cudaStream_t s) {
+  using C = PCfg<BN>;
+  static std::once_flag once[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  cudaError_t ae = cudaSuccess;
+  std::call_once(once[dev & 63], [&] {
+    ae = cudaFuncSetAttribute(program_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              C::kSmem < 118 * 1024 ? 118 * 1024 : C::kSmem);
+  });
+  if (ae != cudaSuccess) return ae;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nct));
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = C::kSmem < 118 * 1024 ? 118 * 1024 : C::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, program_kernel<BN>, reinterpret_cast<const uint8_t*>(ws), status,
+                            kWaitLimitNs);
+}
+
+}  // namespace
+}  // namespace mmf
+
+using namespace mmf;
+
+MMF_EXPORT size_t mmf_program_workspace_bytes(const mmf_projection* p, int n, int64_t T) {
+  Plan P;
+  if (build_plan(p, n, T, 1e-8f, 0, sm_count(), P) != MMF_OK) return 0;
+  return P.bytes;
+}
+
+MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T, float eps,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  if (!(eps > 0.0f) || eps != eps || eps > 1.0f) return MMF_ERR_INVALID_ARG;
+  mmf_status st = validate(p, n, T);
+  if (st != MMF_OK) return st;
+  if (!ws) return MMF_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MMF_ERR_ALIGNMENT;
+  const int nct = sm_count();
+  Plan P;
+  st = build_plan(p, n, T, eps, reinterpret_cast<uintptr_t>(ws), nct, P);
+  if (st != MMF_OK) return st;
+  if (ws_bytes < P.bytes) return MMF_ERR_WORKSPACE;
+  // tensor maps: packed weights (box 64 rows x 32 B, 32-byte swizzle) and activation codes
+  // (box BN rows x 128 B, 128-byte swizzle), exactly as the single-projection kernel
+  P.maps.resize(P.projs.size() + P.ins.size());
+  for (size_t i = 0; i < P.projs.size(); ++i) {
+    const PProj& q = P.projs[i];
+    if (!make_tmap_2d_u8(&P.maps[i], q.Wp, static_cast<uint64_t>(q.K / 4), static_cast<uint64_t>(q.N),
+                         static_cast<uint64_t>(q.K / 4), kPWRow, 64, CU_TENSOR_MAP_SWIZZLE_32B))
+      return MMF_ERR_CUDA;
+  }
+  for (size_t k = 0; k < P.ins.size(); ++k) {
+    const PIn& in = P.ins[k];
+    if (!make_tmap_2d_u8(&P.maps[P.projs.size() + k], in.A, static_cast<uint64_t>(in.K),
+                         static_cast<uint64_t>(T), static_cast<uint64_t>(in.K), kPKB,
+                         static_cast<uint32_t>(P.BN), CU_TENSOR_MAP_SWIZZLE_128B))
+      return MMF_ERR_CUDA;
+  }
+  // host image of the plan region, copied in one stream-ordered copy; counters zeroed
+  const size_t plan_end = static_cast<size_t>(P.h.off_levelctr) + (2 * kMaxLevels + 2) * 4;
+  std::vector<uint8_t> img(plan_end, 0);
+  std::memcpy(img.data(), &P.h, sizeof(PHeader));
+  std::memcpy(img.data() + P.h.off_in, P.ins.data(), P.ins.size() * sizeof(PIn));
+  std::memcpy(img.data() + P.h.off_proj, P.projs.data(), P.projs.size() * sizeof(PProj));
+  std::memcpy(img.data() + P.h.off_units, P.units.data(), P.units.size() * sizeof(PUnit));
+  std::memcpy(img.data() + P.h.off_ctaoff, P.ctaoff.data(), P.ctaoff.size() * sizeof(int32_t));
+  std::memcpy(img.data() + P.h.off_maps, P.maps.data(), P.maps.size() * sizeof(CUtensorMap));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // pageable source: the copy has consumed the host buffer when cudaMemcpyAsync returns
+  if (cudaMemcpyAsync(ws, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MMF_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_runs_mu);
+    g_runs[ws] = RunInfo{P.BN, nct};
+  }
+  return MMF_OK;
+}
+
+MMF_EXPORT mmf_status mmf_program_run(void* ws, void* stream) {
+  if (!ws) return MMF_ERR_INVALID_ARG;
+  RunInfo ri;
+  {
+    std::lock_guard<std::mutex> lk(g_runs_mu);
+    auto it = g_runs.find(ws);
+    if (it == g_runs.end()) return MMF_ERR_INVALID_ARG;
+    ri = it->second;
+  }
+  unsigned* status = device_status_word();
+  if (!status) return MMF_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (ri.BN == 16)
+    e = launch_program<16>(ws, ri.nct, status, s);
+  else if (ri.BN == 32)
+    e = launch_program<32>(ws, ri.nct, status, s);
+  else
+    e = launch_program<64>(ws, ri.nct, status, s);
+  return e == cudaSuccess ? MMF_OK : MMF_ERR_CUDA;
+}
