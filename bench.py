@@ -3,7 +3,12 @@
 
 One step = every FusedBitLinear projection of the workload's layers applied to one batch of T
 tokens: per layer i/f/g_proj (input x_attn), o_proj (x_o), gate_proj with the SiLU-GLU
-epilogue (x_mlp) and down_proj fed by gate_proj's GLU output h.  Each projection is the full
+epilogue (x_mlp) and down_proj fed by gate_proj's GLU output h.  The default data flow
+("path") chains only what this path itself links, gate_proj's GLU output into down_proj; the
+layer's other inputs come from the recurrence, the residual stream and the norms, which are
+outside the path, so they are seeded synthetic activations, one set per layer.  "--dataflow
+chained" instead feeds every projection from an earlier one (o from g, gate from o, the next
+layer from down), the dependency depth of a real layer-by-layer decode.  Each projection is the full
 forward: RMSNorm + int8 activation quantisation, then the tcgen05 ternary contraction with
 the dequantisation epilogue.  Weights are quantised and packed once before timing (the
 offline step of the method); packed weights rotate over enough distinct copies that every
@@ -58,6 +63,8 @@ def parse_args(argv=None):
                     help="target host time of the CPU-baseline sample")
     ap.add_argument("--path", choices=["auto", "program", "launches"], default="auto",
                     help="one program launch per step (decode, T <= 64) or per-projection launches")
+    ap.add_argument("--dataflow", choices=sorted(DATAFLOWS), default="path",
+                    help="which projections feed which (see the module docstring)")
     return ap.parse_args(argv)
 
 
@@ -191,31 +198,53 @@ def quant_bytes(p, T, in_bytes=2):
 
 def step_bytes(wl):
     """Algorithmic HBM bytes of one step run as one program launch: every projection's packed
-    weights, its input read once (fp16) and its output written once; the int8 codes are an
-    on-chip/L2 intermediate."""
+    weights, each distinct input read once (fp16) and each output written once; the int8 codes
+    are an on-chip/L2 intermediate.  Both data flows have, per layer, three distinct inputs of
+    width H (shared by i/f/g, then o's, then gate's) and the GLU output of width I (down's)."""
     T, tot = wl.T, 0
+    widths = {}
     for p in wl.projections:
         n_out = p.N // 2 if p.glu else p.N
-        tot += p.N * p.K // 4 + 2 * T * p.K + 2 * T * n_out
+        tot += p.N * p.K // 4 + 2 * T * n_out
+        widths.setdefault(SOURCE_OF.get(p.name, p.name), p.K)
+    tot += sum(2 * T * k for k in widths.values())
     return tot * wl.layers
 
 
-# Data flow of one layer, in dependency order: i/f/g read the layer input; o reads g's output
-# (standing in for the recurrence output); gate reads o's output (standing in for the residual
-# and norm); down reads the GLU output; the next layer reads down's output.
-LEVEL_OF = {"i_proj": 0, "f_proj": 0, "g_proj": 0, "o_proj": 1, "gate_proj": 2, "down_proj": 3,
-            "proj": 0}
+# Which input each projection reads, and the dependency level it runs at, per data flow.
+# "path": i/f/g/o/gate read the layer's synthetic inputs (level 0), down reads the GLU output
+# (level 1).  "chained": i/f/g read the layer input, o reads g's output, gate reads o's
+# output, down reads the GLU output, the next layer reads down's output (4 levels per layer).
+SOURCE_OF = {"i_proj": "x_attn", "f_proj": "x_attn", "g_proj": "x_attn", "proj": "x_attn",
+             "o_proj": "x_o", "gate_proj": "x_mlp", "down_proj": "h"}
+DATAFLOWS = {
+    "path": {"i_proj": 0, "f_proj": 0, "g_proj": 0, "o_proj": 0, "gate_proj": 0,
+             "down_proj": 1, "proj": 0},
+    "chained": {"i_proj": 0, "f_proj": 0, "g_proj": 0, "o_proj": 1, "gate_proj": 2,
+                "down_proj": 3, "proj": 0},
+}
+LEVELS_PER_LAYER = {"path": 2, "chained": 4}   # "path": the layers are independent, so a
+# whole step has 2 levels; "chained": 4 per layer, one after another
+DATAFLOW_TEXT = {
+    "path": ("per layer: i/f/g read x_attn, o reads x_o, gate reads x_mlp (seeded synthetic "
+             "activations, one set per layer: their producers are outside this path); down "
+             "reads gate's GLU output"),
+    "chained": ("per layer: i/f/g read the layer input, o reads g's output, gate reads o's "
+                "output, down reads the GLU output, the next layer reads down's"),
+}
 
 
 class GpuWorkload:
     """Device buffers for one replica: packed weight copies, the step input, per-layer outputs,
     and either one planned program per weight copy (T <= 64) or per-projection launches."""
 
-    def __init__(self, wl, device, path="auto"):
+    def __init__(self, wl, device, path="auto", dataflow="path"):
         import torch
         import ternary_weight_lm_b200 as mmf
         self.torch, self.mmf = torch, mmf
         self.wl, self.dev = wl, device
+        self.dataflow = dataflow
+        self.level_of = DATAFLOWS[dataflow]
         T = wl.T
         H = wl.projections[0].K
         need = 2 * L2_BYTES
@@ -232,9 +261,16 @@ class GpuWorkload:
             n = self.copies * wl.layers
             self.Wp[p.name] = [Wp0] + [Wp0.clone() for _ in range(n - 1)]
             self.beta[p.name] = [b0] + [b0.clone() for _ in range(n - 1)]
-        self.x = torch.from_numpy(synth.activations(0, "x_attn", T, H, dtype=xdt,
-                                                    outlier_frac=wl.outlier_frac,
-                                                    outlier_scale=wl.outlier_scale)).to(device)
+        # step inputs: "path" has one set of synthetic activations per layer and source,
+        # "chained" only the first layer's input
+        srcs = sorted({SOURCE_OF.get(p.name, "x_attn") for p in wl.projections} - {"h"})
+        self.xin = []
+        for l in range(wl.layers if dataflow == "path" else 1):
+            self.xin.append({src: torch.from_numpy(synth.activations(
+                0, src if l == 0 else f"{src}/layer{l}", T, H, dtype=xdt,
+                outlier_frac=wl.outlier_frac, outlier_scale=wl.outlier_scale)).to(device)
+                for src in (srcs if dataflow == "path" else ["x_attn"])})
+        self.x = self.xin[0]["x_attn"]
         self.y = [{p.name: torch.empty((T, p.N // 2 if p.glu else p.N), dtype=self.ydt,
                                        device=device) for p in wl.projections}
                   for _ in range(wl.layers)]
@@ -253,13 +289,20 @@ class GpuWorkload:
 
     def input_of(self, l, p):
         ys = self.y[l]
+        if p.name == "down_proj":
+            return ys["gate_proj"]                  # the GLU output, in both data flows
+        if self.dataflow == "path":
+            return self.xin[l][SOURCE_OF.get(p.name, "x_attn")]
         if p.name in ("i_proj", "f_proj", "g_proj", "proj"):
             return self.x if l == 0 else self.y[l - 1]["down_proj"]
         if p.name == "o_proj":
             return ys["g_proj"]
-        if p.name == "gate_proj":
-            return ys["o_proj"]
-        return ys["gate_proj"]                      # down_proj reads the GLU output
+        return ys["o_proj"]                         # gate_proj
+
+    @property
+    def step_inputs(self):
+        """The device tensors a step reads from outside (copied in from the host in e2e)."""
+        return [t for d in self.xin for _, t in sorted(d.items())]
 
     def projection_list(self, c):
         out = []
@@ -268,7 +311,8 @@ class GpuWorkload:
             for p in self.wl.projections:
                 out.append(dict(x=self.input_of(l, p), Wp=self.Wp[p.name][li],
                                 beta=self.beta[p.name][li], y=self.y[l][p.name], glu=p.glu,
-                                level=4 * l + LEVEL_OF[p.name]))
+                                level=self.level_of[p.name] if self.dataflow == "path" else
+                                LEVELS_PER_LAYER["chained"] * l + self.level_of[p.name]))
         return out
 
     @property
@@ -285,7 +329,7 @@ class GpuWorkload:
         mmf = self.mmf
         for l in range(self.wl.layers):
             li = c * self.wl.layers + l
-            for p in sorted(self.wl.projections, key=lambda q: LEVEL_OF[q.name]):
+            for p in sorted(self.wl.projections, key=lambda q: self.level_of[q.name]):
                 f = mmf.mmf_bitlinear_glu_forward if p.glu else mmf.mmf_bitlinear_forward
                 f(self.input_of(l, p), None, 1e-8, self.Wp[p.name][li], self.beta[p.name][li],
                   p.N, self.y[l][p.name], self.ws)
@@ -304,7 +348,7 @@ class GpuWorkload:
         T = self.wl.T
         for l in range(self.wl.layers):
             li = c * self.wl.layers + l
-            for p in sorted(self.wl.projections, key=lambda q: LEVEL_OF[q.name]):
+            for p in sorted(self.wl.projections, key=lambda q: self.level_of[q.name]):
                 A = self.A.view(-1)[:T * p.K].view(T, p.K)
                 e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 e0.record()
@@ -346,7 +390,7 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device(f"cuda:{local_rank}")
     wl = synth.WORKLOADS[args.workload]
-    g = GpuWorkload(wl, dev, args.path)
+    g = GpuWorkload(wl, dev, args.path, args.dataflow)
     stream = torch.cuda.Stream(device=dev)
     T = wl.T
 
@@ -462,9 +506,9 @@ def run_gpu(args, rank, world, local_rank):
     # ---- e2e: the public API with host buffers, copies inside the timed region
     e2e = None
     if not args.no_e2e:
-        hx = g.x.cpu().pin_memory()
+        hxs = [t.cpu().pin_memory() for t in g.step_inputs]
         hy = torch.empty_like(g.final_output, device="cpu").pin_memory()
-        h2d = hx.numel() * hx.element_size()
+        h2d = sum(t.numel() * t.element_size() for t in hxs)
         d2h = hy.numel() * hy.element_size()
         e2e_steps = min(args.steps, 200)
         with torch.cuda.stream(stream):
@@ -476,7 +520,8 @@ def run_gpu(args, rank, world, local_rank):
         with torch.cuda.stream(stream):
             s0.record()
             for i in range(e2e_steps):
-                g.x.copy_(hx, non_blocking=True)
+                for dst, src in zip(g.step_inputs, hxs):
+                    dst.copy_(src, non_blocking=True)
                 g.run_step(i)
                 hy.copy_(g.final_output, non_blocking=True)
             s1.record()
@@ -488,7 +533,7 @@ def run_gpu(args, rank, world, local_rank):
                "steps": e2e_steps,
                "path": ("mmf_program_run (one launch per step)" if g.use_program else
                         "mmf_bitlinear_forward / _glu_forward per projection") +
-                       ", step input from pinned host memory, last output back to pinned host"}
+                       ", step inputs from pinned host memory, last output back to pinned host"}
 
     return {
         "value": value, "ms_per_step": ms_per_step, "elapsed_s": elapsed_s, "clocks": clocks,
@@ -509,38 +554,43 @@ def capture_one(g, stream, j):
 
 
 # ----------------------------------------------------------------------------- oracle arm
-def oracle_sample(wl, n_tokens):
+def oracle_sample(wl, n_tokens, dataflow="path"):
     """Inputs of a bounded sample of one step for the oracle: the first n_tokens tokens of the
-    step input and one layer's weights, quantised by the oracle itself."""
+    first layer's step inputs (the same seeded activations as the GPU arm's) and one layer's
+    weights, quantised by the oracle itself."""
     import oracle
     H = wl.projections[0].K
-    x = synth.activations(0, "x_attn", wl.T, H, dtype=np.float32 if wl.x_dtype == "f32"
-                          else np.float16, outlier_frac=wl.outlier_frac,
-                          outlier_scale=wl.outlier_scale)[:n_tokens]
+    xdt = np.float32 if wl.x_dtype == "f32" else np.float16
+    srcs = sorted({SOURCE_OF.get(p.name, "x_attn") for p in wl.projections} - {"h"})
+    xs = {src: synth.activations(0, src, wl.T, H, dtype=xdt, outlier_frac=wl.outlier_frac,
+                                 outlier_scale=wl.outlier_scale)[:n_tokens]
+          for src in (srcs if dataflow == "path" else ["x_attn"])}
     weights = {}
     for p in wl.projections:
         W = synth.weights(0, p.name, p.N, p.K)
         beta = oracle.absmean_beta(W)
         weights[p.name] = (oracle.ternary_codes(W, beta), beta)
-    return x, weights
+    return xs, weights
 
 
-def oracle_step(wl, x, weights):
-    """One layer of the step in the same data flow as the GPU arm (i/f/g on the input, o on
-    g's output, gate on o's output, down on the GLU output), outputs rounded to the output
+def oracle_step(wl, xs, weights, dataflow="path"):
+    """One layer of the step in the same data flow as the GPU arm, outputs rounded to the output
     dtype where they feed the next projection."""
     import oracle
     ydt = np.float32 if wl.y_dtype == "f32" else np.float16
+    level_of = DATAFLOWS[dataflow]
     outs = {}
-    for p in sorted(wl.projections, key=lambda q: LEVEL_OF[q.name]):
-        if p.name in ("i_proj", "f_proj", "g_proj", "proj"):
-            xin = x
+    for p in sorted(wl.projections, key=lambda q: level_of[q.name]):
+        if p.name == "down_proj":
+            xin = outs["gate_proj"]
+        elif dataflow == "path":
+            xin = xs[SOURCE_OF.get(p.name, "x_attn")]
+        elif p.name in ("i_proj", "f_proj", "g_proj", "proj"):
+            xin = xs["x_attn"]
         elif p.name == "o_proj":
             xin = outs["g_proj"]
-        elif p.name == "gate_proj":
-            xin = outs["o_proj"]
         else:
-            xin = outs["gate_proj"]
+            xin = outs["o_proj"]
         c, beta = weights[p.name]
         q, gamma, _ = oracle.rmsnorm_actquant(xin)
         y = oracle.dequant(oracle.ternary_accumulate(q, c), gamma, beta)
@@ -550,15 +600,15 @@ def oracle_step(wl, x, weights):
     return outs
 
 
-def oracle_tokens_per_s(wl, seconds, n_tokens=None):
+def oracle_tokens_per_s(wl, seconds, n_tokens=None, dataflow="path"):
     """Time the oracle on bounded samples for about `seconds` of host time."""
     if n_tokens is None:
         n_tokens = min(wl.T, 8)
-    xs, weights = oracle_sample(wl, n_tokens)
-    oracle_step(wl, xs, weights)                 # warm
+    xs, weights = oracle_sample(wl, n_tokens, dataflow)
+    oracle_step(wl, xs, weights, dataflow)       # warm
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(wl, xs, weights)
+        oracle_step(wl, xs, weights, dataflow)
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -567,7 +617,7 @@ def oracle_tokens_per_s(wl, seconds, n_tokens=None):
     tps = n_tokens * reps / el / wl.layers
     return tps, {"kind": "oracle", "cores": 1,
                  "sample": f"first {n_tokens} of {wl.T} tokens through all "
-                           f"{len(wl.projections)} chained projections of one layer, repeated "
+                           f"{len(wl.projections)} projections of one layer ({dataflow} data flow), repeated "
                            f"{reps} times ({el:.1f} s); tokens/s scaled by 1/{wl.layers} "
                            f"layers", "value": round(tps, 3), "unit": "tokens/s"}
 
@@ -577,17 +627,18 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     # size each step so that warm-up + K steps stay within about two minutes
-    xs, weights = oracle_sample(wl, 1)
+    df = args.dataflow
+    xs, weights = oracle_sample(wl, 1, df)
     t0 = time.perf_counter()
-    oracle_step(wl, xs, weights)
+    oracle_step(wl, xs, weights, df)
     per_token_layer = time.perf_counter() - t0
     n_tok = int(max(1, min(wl.T, 120.0 / max(1, args.steps + args.warmup) / per_token_layer)))
-    xs, weights = oracle_sample(wl, n_tok)
+    xs, weights = oracle_sample(wl, n_tok, df)
     for _ in range(args.warmup):
-        oracle_step(wl, xs, weights)
+        oracle_step(wl, xs, weights, df)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(wl, xs, weights)
+        oracle_step(wl, xs, weights, df)
     el = time.perf_counter() - t0
     tps = n_tok * args.steps / el / wl.layers
     cpu = {"kind": "oracle", "cores": 1, "value": round(tps, 3), "unit": "tokens/s",
@@ -597,23 +648,22 @@ def run_reference(args, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": config_of(wl, None), "cpu_baseline": cpu,
+            "config": config_of(wl, None, df), "cpu_baseline": cpu,
             "e2e": {"value": round(tps, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
-def config_of(wl, res):
+def config_of(wl, res, dataflow="path"):
     c = {"workload": wl.name, "tokens_per_step": wl.T, "layers_per_step": wl.layers,
          "projections": ",".join(p.name + ("(glu)" if p.glu else "") for p in wl.projections),
-         "x_dtype": wl.x_dtype, "y_dtype": wl.y_dtype, "parallelism": "replicas"}
+         "x_dtype": wl.x_dtype, "y_dtype": wl.y_dtype, "parallelism": "replicas",
+         "dataflow": DATAFLOW_TEXT[dataflow]}
     if res is not None:
         c["weight_copies"] = res["copies"]
         c["l2"] = ("packed weights rotate over %d distinct copies (%.0f MB > 2x L2); "
                    "activations stay L2-resident as in a layer-by-layer decode"
                    % (res["copies"], res["copies"] * wl.packed_bytes_per_layer * wl.layers / 1e6))
         c["timing"] = "CUDA graph replays of whole steps, CUDA events on the launch stream"
-        c["dataflow"] = ("per layer: i/f/g read the layer input, o reads g's output, gate reads "
-                         "o's output, down reads the GLU output, the next layer reads down's")
     return c
 
 
@@ -642,7 +692,7 @@ def main(argv=None):
                     "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                     "ms_per_step": round(res["ms_per_step"], 6), "higher_is_better": True,
                     "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-                    "data": "synthetic", "config": config_of(wl, res),
+                    "data": "synthetic", "config": config_of(wl, res, args.dataflow),
                     "weight_gbs": round(res["weight_gbs"], 1),
                     "int8_tops": round(res["int8_tops"], 2),
                     "path": res["path"],
@@ -651,7 +701,8 @@ def main(argv=None):
                     "gpu_launches": res["launches"],
                 }
                 if not args.no_cpu_baseline and world == 1:
-                    _, cpu = oracle_tokens_per_s(wl, args.cpu_seconds)
+                    _, cpu = oracle_tokens_per_s(wl, args.cpu_seconds,
+                                                 dataflow=args.dataflow)
                     line["cpu_baseline"] = cpu
                 else:
                     line["cpu_baseline"] = None

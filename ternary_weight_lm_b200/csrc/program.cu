@@ -41,18 +41,28 @@
 namespace mmf {
 namespace {
 
-constexpr int kPThreads = 192;
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 unpack, 6-9 quantise + epilogue.
+constexpr int kPThreads = 320;
 constexpr int kPEpi = 128;
-constexpr int kPKB = 128;                  // K per stage
-constexpr int kPWRow = kPKB / 4;           // packed bytes per weight row per stage
-constexpr int kPWStage = 128 * kPWRow;     // 4 KB
-constexpr int kPStages = 12;               // SMEM stages == TMEM slots
+constexpr int kPEpiT0 = 192;               // first epilogue thread
+constexpr int kPKB = 128;                  // K per TMEM slot (one sub-block)
+constexpr int kPSub = 4;                   // sub-blocks per shared-memory stage
+constexpr int kPKS = kPKB * kPSub;         // K per stage (512)
+constexpr int kPWRow = kPKS / 4;           // packed bytes per weight row per stage: 128
+constexpr int kPWStage = 128 * kPWRow;     // 16 KB: one 128-byte line of each of 128 rows
+constexpr int kPSlots = 12;                // TMEM A slots of one sub-block each
+constexpr int kPGroups = kPSlots / kPSub;  // slot groups: stage counter c writes group c % 3
 constexpr int kPACol0 = 128;               // TMEM: accumulators at 0 and 64, slots from 128
 constexpr int kMaxLevels = 128;
 constexpr int kMaxProj = 1024;
 constexpr int kMaxSplit = 16;
 constexpr int kMinSplitKb = 8;             // latency beats spreading at decode sizes
 constexpr uint64_t kPDrainNs = 2000000000ull;
+static_assert(kPACol0 + kPSlots * 32 == 512, "TMEM columns");
+// Two partial accumulators per unit (even / odd sub-blocks) when they fit in the unit's 64
+// accumulator columns.
+template <int BN>
+constexpr bool kSplitAcc = BN <= 32;
 
 struct PProj {
   const uint8_t* Wp;
@@ -84,15 +94,22 @@ struct PHeader {
 
 template <int BN>
 struct PCfg {
-  static constexpr int kAct = BN * kPKB;
+  static constexpr int kActSub = BN * kPKB;       // activation codes of one sub-block
+  static constexpr int kAct = kPSub * kActSub;
   static constexpr int kStage = kAct + kPWStage;
-  static constexpr int kBar = (8 * (3 * kPStages + 5) + 127) / 128 * 128;   // keeps what follows 128-byte aligned
-  static constexpr int kXbuf = BN * 64 * 4;      // GLU exchange: multiplier half, fp32
-  static constexpr int kTok = 8 * 64;            // per-token scale and code sum
-  static constexpr int kOst = BN * 128 * 2;      // fp16 output staging [token][column]
-  static constexpr int kSmem = 1024 + kPStages * kStage + kBar + kXbuf + kTok + kOst + 64;
-  static_assert(kSmem <= 227 * 1024, "shared memory");
-  static_assert(kSmem >= 118 * 1024 || BN < 64, "one CTA per SM");
+  static constexpr int kCh = 16;                  // epilogue chunk: tokens per TMEM load
+  static constexpr int kXbuf = kCh * 64 * 4;      // GLU exchange: multiplier half, fp32
+  static constexpr int kTok = 8 * 64;             // per-token scale and code sum
+  static constexpr int kOst = BN * 128 * 2;       // fp16 output staging [token][column]
+  static constexpr int kFixed = 1024 + 1024 + kXbuf + kTok + kOst + 64;
+  static constexpr int kStagesFit = (227 * 1024 - 512 - kFixed) / kStage;
+  static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
+  static constexpr int kBar = (8 * (2 * kStages + kPGroups + 5) + 127) / 128 * 128;
+  static constexpr int kSmem = 1024 + kStages * kStage + kBar + kXbuf + kTok + kOst + 64;
+  static_assert(kStages >= 3, "pipeline depth");
+  static_assert(kBar <= 1024, "barrier area");
+  static_assert(kSmem <= 227 * 1024 - 512, "shared memory");
+  static_assert(kSmem >= 118 * 1024, "one CTA per SM");
 };
 
 // ------------------------------------------------------------------------------ device helpers
@@ -244,6 +261,122 @@ __device__ void quant_row(const PIn in, int t, float eps, int et, double* red_d,
   named_bar_sync(1, kPEpi);   // the scratch is reused by the next row
 }
 
+// One warp quantises row t of input `in` alone, with the same operations per element as
+// quant_row (only the order in which the per-lane sums of squares are added differs, which can
+// move the double sum by an ulp, far below the float rounding of the mean).  Used when a level
+// has more rows than CTAs, so that each CTA's four epilogue warps work on four rows at once.
+// The row is streamed kQW vectors of 16 bytes per lane at a time (any K; few registers, as
+// the kernel's ten warps leave 168 per thread), in passes over L2:
+//   1. sum of squares (double) and, without a norm weight, max|x|;
+//   2. only with a norm weight: gamma = max |(x*inv)*g| element by element;
+//   3. the codes.
+// Without a norm weight gamma = (max|x|)*inv exactly: rounding is monotone, so the largest
+// |x*inv| comes from the largest |x| (and *1.0f is exact).
+constexpr int kQW = 2;
+__device__ void quant_row_warp(const PIn in, int t, float eps, int lane) {
+  const int K = in.K;
+  const int E = in.xdt == kInF16 ? 8 : 4;
+  const int nvec = K / E;
+  const uint4* xr = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(in.x) +
+                                                   static_cast<int64_t>(t) * K * (E == 8 ? 2 : 4));
+  double ss = 0.0;
+  float mx = 0.0f;
+#pragma unroll 1
+  for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
+    uint4 raw[kQW];
+#pragma unroll
+    for (int i = 0; i < kQW; ++i) {
+      const int vi = v0 + lane + 32 * i;
+      if (vi < nvec) raw[i] = __ldcg(xr + vi);
+    }
+#pragma unroll
+    for (int i = 0; i < kQW; ++i) {
+      if (v0 + lane + 32 * i < nvec) {
+        float v[8];
+        int n;
+        widen16(raw[i], in.xdt, v, n);
+        for (int e = 0; e < n; ++e) {
+          const double d = static_cast<double>(v[e]);
+          ss = __fma_rn(d, d, ss);
+          mx = fmaxf(mx, fabsf(v[e]));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
+  const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+  float amax = 0.0f;
+  if (in.g == nullptr) {
+    amax = __fmul_rn(mx, inv_r);
+  } else {
+  #pragma unroll 1
+  for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
+      uint4 raw[kQW];
+#pragma unroll
+      for (int i = 0; i < kQW; ++i) {
+        const int vi = v0 + lane + 32 * i;
+        if (vi < nvec) raw[i] = __ldcg(xr + vi);
+      }
+#pragma unroll
+      for (int i = 0; i < kQW; ++i) {
+        const int vi = v0 + lane + 32 * i;
+        if (vi < nvec) {
+          float v[8];
+          int n;
+          widen16(raw[i], in.xdt, v, n);
+          for (int e = 0; e < n; ++e)
+            amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), __ldg(in.g + vi * E + e))));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float gm = fmaxf(amax, 1e-5f);
+  const float s = __fdiv_rn(127.0f, gm);
+  int rs = 0;
+  int8_t* ar = in.A + static_cast<int64_t>(t) * K;
+#pragma unroll 1
+  for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
+    uint4 raw[kQW];
+#pragma unroll
+    for (int i = 0; i < kQW; ++i) {
+      const int vi = v0 + lane + 32 * i;
+      if (vi < nvec) raw[i] = __ldcg(xr + vi);
+    }
+#pragma unroll
+    for (int i = 0; i < kQW; ++i) {
+      const int vi = v0 + lane + 32 * i;
+      if (vi < nvec) {
+        float v[8];
+        int n;
+        widen16(raw[i], in.xdt, v, n);
+        uint32_t wd[2] = {0u, 0u};
+        for (int e = 0; e < n; ++e) {
+          const float gk = in.g ? __ldg(in.g + vi * E + e) : 1.0f;
+          const float xh = __fmul_rn(__fmul_rn(v[e], inv_r), gk);
+          int q = __float2int_rn(__fmul_rn(xh, s));
+          q = max(-128, min(127, q));
+          rs += q;
+          wd[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (e & 3));
+        }
+        if (E == 8)
+          *reinterpret_cast<uint2*>(ar + vi * 8) = make_uint2(wd[0], wd[1]);
+        else
+          *reinterpret_cast<uint32_t*>(ar + vi * 4) = wd[0];
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+  if (lane == 0) {
+    in.gamma[t] = gm;
+    in.rowsum[t] = rs;
+  }
+}
+
 __device__ __forceinline__ void unpack_word4(uint32_t w, uint32_t* out) {
   out[0] = w & 0x03030303u;
   out[1] = (w >> 2) & 0x03030303u;
@@ -251,78 +384,111 @@ __device__ __forceinline__ void unpack_word4(uint32_t w, uint32_t* out) {
   out[3] = (w >> 6) & 0x03030303u;
 }
 
-// Dequantise (and GLU) one finished tile held as int32 sums acc[j] (token j, tile row r).
-// tsc/trs: per-token scale (gamma/127 * beta) and code sum, staged in shared memory.
-// fp16 outputs go through ostage ([token][column] fp16) so that each token's 128 (or 64 GLU)
-// outputs leave as 16-byte stores; fp32 outputs are stored directly.
-template <int BN>
-__device__ __forceinline__ void finalize_tile(const PProj pj, int tile, int T,
-                                              const int32_t (&acc)[BN], int r,
-                                              const float* __restrict__ tsc,
-                                              const int32_t* __restrict__ trs,
-                                              float* __restrict__ xbuf,
-                                              __half* __restrict__ ostage) {
-  const int et = threadIdx.x - 64;
-  // pass 1 (loads and arithmetic only, so the 64 independent tokens overlap): dequantised
-  // values of this thread's row in registers
-  float v[BN];
-#pragma unroll
-  for (int j = 0; j < BN; ++j) v[j] = j < T ? static_cast<float>(acc[j] - trs[j]) * tsc[j] : 0.0f;
+// Dequantise (and GLU) tokens c0 .. c0+CH-1 of a finished tile, held as int32 sums v[jj]
+// (token c0+jj, tile row r).  tsc/trs: per-token scale (gamma/127 * beta) and code sum, staged
+// in shared memory.  fp16 results go to ostage ([token][column] fp16, written out by
+// store_tile); fp32 results are stored directly.  The GLU pairs row r < 64 (gated half) with
+// row r + 64 (multiplier) through xbuf.
+template <int CH>
+__device__ __forceinline__ void finalize_chunk(const PProj& pj, int tile, int T, int c0,
+                                               const int32_t (&v)[CH], int r,
+                                               const float* __restrict__ tsc,
+                                               const int32_t* __restrict__ trs,
+                                               float* __restrict__ xbuf,
+                                               __half* __restrict__ ostage) {
   if (!pj.glu) {
     if (pj.ydt == MMF_F16) {
 #pragma unroll
-      for (int j = 0; j < BN; ++j)
-        if (j < T) ostage[j * 128 + r] = __float2half_rn(v[j]);
-      named_bar_sync(1, kPEpi);
-      // T rows of 128 fp16 = 16 chunks of 16 bytes per row
-      for (int c = et; c < T * 16; c += kPEpi) {
-        const int j = c >> 4, k8 = (c & 15) * 8;
-        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(pj.y) + static_cast<int64_t>(j) * pj.N +
-                                  static_cast<int64_t>(tile) * 128 + k8) =
-            *reinterpret_cast<const uint4*>(ostage + j * 128 + k8);
+      for (int jj = 0; jj < CH; ++jj) {
+        const int j = c0 + jj;
+        if (j < T)
+          ostage[j * 128 + r] = __float2half_rn(static_cast<float>(v[jj] - trs[j]) * tsc[j]);
       }
     } else {
       const int64_t n = static_cast<int64_t>(tile) * 128 + r;
 #pragma unroll
-      for (int j = 0; j < BN; ++j)
-        if (j < T) reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * pj.N + n] = v[j];
+      for (int jj = 0; jj < CH; ++jj) {
+        const int j = c0 + jj;
+        if (j < T)
+          reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * pj.N + n] =
+              static_cast<float>(v[jj] - trs[j]) * tsc[j];
+      }
+    }
+    return;
+  }
+  if (r >= 64) {
+#pragma unroll
+    for (int jj = 0; jj < CH; ++jj) {
+      const int j = c0 + jj;
+      xbuf[jj * 64 + (r - 64)] = j < T ? static_cast<float>(v[jj] - trs[j]) * tsc[j] : 0.0f;
+    }
+  }
+  named_bar_sync(1, kPEpi);
+  if (r < 64) {
+    const int64_t I = pj.N / 2;
+#pragma unroll
+    for (int jj = 0; jj < CH; ++jj) {
+      const int j = c0 + jj;
+      if (j < T) {
+        const float g = static_cast<float>(v[jj] - trs[j]) * tsc[j];
+        const float h = __fdividef(g, 1.0f + expf(-g)) * xbuf[jj * 64 + r];
+        if (pj.ydt == MMF_F16)
+          ostage[j * 64 + r] = __float2half_rn(h);
+        else
+          reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * I + static_cast<int64_t>(tile) * 64 + r] = h;
+      }
+    }
+  }
+  named_bar_sync(1, kPEpi);   // xbuf is reused by the next chunk
+}
+
+// fp16 outputs leave ostage as 16-byte stores: T rows of 128 (or 64 for the GLU) columns.
+__device__ __forceinline__ void store_tile(const PProj& pj, int tile, int T, int et,
+                                           const __half* __restrict__ ostage) {
+  if (pj.ydt != MMF_F16) return;
+  named_bar_sync(1, kPEpi);
+  if (!pj.glu) {
+    for (int c = et; c < T * 16; c += kPEpi) {
+      const int j = c >> 4, k8 = (c & 15) * 8;
+      *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(pj.y) + static_cast<int64_t>(j) * pj.N +
+                                static_cast<int64_t>(tile) * 128 + k8) =
+          *reinterpret_cast<const uint4*>(ostage + j * 128 + k8);
     }
   } else {
-    // rows 0-63 of the tile are the gated half, rows 64-127 the multiplier half
-    if (r >= 64) {
-#pragma unroll
-      for (int j = 0; j < BN; ++j)
-        if (j < T) xbuf[j * 64 + (r - 64)] = v[j];
-    }
-    named_bar_sync(1, kPEpi);
     const int64_t I = pj.N / 2;
-    if (r < 64) {
-      float u[BN];
-#pragma unroll
-      for (int j = 0; j < BN; ++j) u[j] = j < T ? xbuf[j * 64 + r] : 0.0f;
-#pragma unroll
-      for (int j = 0; j < BN; ++j) v[j] = __fdividef(v[j], 1.0f + expf(-v[j])) * u[j];
-      if (pj.ydt == MMF_F16) {
-#pragma unroll
-        for (int j = 0; j < BN; ++j)
-          if (j < T) ostage[j * 64 + r] = __float2half_rn(v[j]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < BN; ++j)
-          if (j < T)
-            reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * I + static_cast<int64_t>(tile) * 64 + r] = v[j];
-      }
+    for (int c = et; c < T * 8; c += kPEpi) {
+      const int j = c >> 3, k8 = (c & 7) * 8;
+      *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(pj.y) + static_cast<int64_t>(j) * I +
+                                static_cast<int64_t>(tile) * 64 + k8) =
+          *reinterpret_cast<const uint4*>(ostage + j * 64 + k8);
     }
-    named_bar_sync(1, kPEpi);
-    if (pj.ydt == MMF_F16) {
-      // T rows of 64 fp16 = 8 chunks of 16 bytes per row
-      for (int c = et; c < T * 8; c += kPEpi) {
-        const int j = c >> 3, k8 = (c & 7) * 8;
-        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(pj.y) + static_cast<int64_t>(j) * I +
-                                  static_cast<int64_t>(tile) * 64 + k8) =
-            *reinterpret_cast<const uint4*>(ostage + j * 64 + k8);
-      }
-    }
+  }
+}
+
+// Loads CH accumulator columns at taddr and, when `two`, adds the partial sum held 32 columns
+// further on.
+template <int CH>
+__device__ __forceinline__ void load_acc(uint32_t taddr, int32_t (&v)[CH]) {
+  uint32_t u[32];
+  if constexpr (CH == 16) {
+    tc_ld_32x32b_x16(taddr, u);
+  } else {
+    static_assert(CH == 32, "chunk");
+    tc_ld_32x32b_x32(taddr, u);
+  }
+  tc_wait_ld();
+#pragma unroll
+  for (int j = 0; j < CH; ++j) v[j] = static_cast<int32_t>(u[j]);
+}
+
+template <int CH>
+__device__ __forceinline__ void load_acc_sum(uint32_t taddr, bool two, int32_t (&v)[CH]) {
+  load_acc<CH>(taddr, v);
+  if (two) {
+    int32_t w[CH];
+    load_acc<CH>(taddr + 32u, w);
+#pragma unroll
+    for (int j = 0; j < CH; ++j) v[j] += w[j];
   }
 }
 
@@ -330,12 +496,13 @@ template <int BN>
 __global__ void __launch_bounds__(kPThreads, 1)
 program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_ns) {
   using C = PCfg<BN>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* s_act = smem;
-  uint8_t* s_w = smem + kPStages * C::kAct;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + kPStages * kPWStage);
+  uint8_t* s_act = smem;                              // S stages of kAct (1024-aligned)
+  uint8_t* s_w = smem + S * C::kAct;                  // S stages of 16 KB (1024-aligned)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_w + S * kPWStage);
   float* xbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + C::kBar);
   float* tsc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(xbuf) + C::kXbuf);
   int32_t* trs = reinterpret_cast<int32_t*>(tsc + 64);
@@ -348,20 +515,27 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   __shared__ float s_red_f[4];
   __shared__ int s_red_i[4];
 
-  auto full = [&](int s) { return smem_u32(bars + s); };
-  auto afull = [&](int s) { return smem_u32(bars + kPStages + s); };
-  auto empty = [&](int s) { return smem_u32(bars + 2 * kPStages + s); };
-  auto accfull = [&](int b) { return smem_u32(bars + 3 * kPStages + b); };
-  auto accempty = [&](int b) { return smem_u32(bars + 3 * kPStages + 2 + b); };
-  const uint32_t drainbar = smem_u32(bars + 3 * kPStages + 4);
+  // Stage counter c (per CTA, over all its units) uses shared-memory stage c % S and TMEM slot
+  // group c % 3 (four slots, one per sub-block).  full(s): stage s's weight line and activation
+  // sub-tiles landed.  empty(s): the unpack warps read its weights and the MMAs of that stage
+  // completed -- one commit per stage, which also tells the unpack warps that the stage's slot
+  // group is free again (commits are costly on the MMA pipe, so there is no per-slot signal).
+  // afull(g): the unpack warps wrote slot group g.  accfull/accempty(b): accumulator b finished /
+  // read by the epilogue.
+  auto full = [&](int st) { return smem_u32(bars + st); };
+  auto empty = [&](int st) { return smem_u32(bars + S + st); };
+  auto afull = [&](int gi) { return smem_u32(bars + 2 * S + gi); };
+  auto accfull = [&](int b) { return smem_u32(bars + 2 * S + kPGroups + b); };
+  auto accempty = [&](int b) { return smem_u32(bars + 2 * S + kPGroups + 2 + b); };
+  const uint32_t drainbar = smem_u32(bars + 2 * S + kPGroups + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kPStages; ++s) {
-      mbar_init(full(s), 1);
-      mbar_init(afull(s), 4);
-      mbar_init(empty(s), 1 + 4);
+    for (int st = 0; st < S; ++st) {
+      mbar_init(full(st), 1);
+      mbar_init(empty(st), 1 + 4);
     }
+    for (int gi = 0; gi < kPGroups; ++gi) mbar_init(afull(gi), 4);
     for (int b = 0; b < 2; ++b) {
       mbar_init(accfull(b), 1);
       mbar_init(accempty(b), 4);
@@ -400,6 +574,9 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
+    // A stage is up to four k-blocks of one unit: one 128-byte line of each of the tile's 128
+    // packed weight rows (two boxes of 64 rows) and one activation sub-tile per k-block.  The
+    // weights run ahead of the activations (they do not depend on them), up to a full ring.
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_a = l2_policy_evict_last();
@@ -437,8 +614,8 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       int q_level = -1;
       bool ok = true;
       while (ok && ac.ui < u_end) {
-        // 1. the activation tile of every stage whose weights are already requested (the
-        //    weights ran ahead); at a new level, first wait until its codes exist
+        // 1. the activation sub-tiles of every stage whose weights are already requested; at a
+        //    new level, first wait until its codes exist
         while (ai < wi) {
           if (ac.level > q_level) {
             if (!grid_wait(lvl + 2 * ac.level, static_cast<unsigned>(nct), poison, limit_ns,
@@ -450,122 +627,218 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
             fence_proxy_async_global();
             q_level = ac.level;
           }
-          const int s = static_cast<int>(ai % kPStages);
-          tma_load_2d(smem_u32(s_act + s * C::kAct), ac.amap, full(s), (ac.kb0 + ac.k) * kPKB, 0,
-                      pol_a);
+          const int st = static_cast<int>(ai % S);
+          const int nsub = min(kPSub, ac.nkb - ac.k);
+          for (int i = 0; i < nsub; ++i)
+            tma_load_2d(smem_u32(s_act + st * C::kAct + i * C::kActSub), ac.amap, full(st),
+                        (ac.kb0 + ac.k + i) * kPKB, 0, pol_a);
           ++ai;
-          if (++ac.k == ac.nkb) load_cur(ac, ac.ui + 1);
+          ac.k += kPSub;
+          if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
         }
         if (!ok || wc.ui >= u_end) continue;
-        // 2. the packed weights of the next stage, up to a full ring ahead (they do not depend
-        //    on any activation)
-        const int s = static_cast<int>(wi % kPStages);
-        if (wi >= kPStages &&
-            !mbar_wait_bounded(empty(s), static_cast<uint32_t>(((wi / kPStages) - 1) & 1),
-                               limit_ns, abort_flag, status)) {
+        // 2. the packed weights of the next stage
+        const int st = static_cast<int>(wi % S);
+        if (wi >= S &&
+            !mbar_wait_bounded(empty(st), static_cast<uint32_t>(((wi / S) - 1) & 1), limit_ns,
+                               abort_flag, status)) {
           ok = false;
           break;
         }
-        const int kg = wc.kb0 + wc.k;
-        mbar_arrive_expect_tx(full(s), C::kStage);
-        uint8_t* wdst = s_w + s * kPWStage;
-        tma_load_2d(smem_u32(wdst), wc.wmap, full(s), kg * kPWRow, wc.r0, pol_w);
-        tma_load_2d(smem_u32(wdst + kPWStage / 2), wc.wmap, full(s), kg * kPWRow, wc.r1, pol_w);
+        const int nsub = min(kPSub, wc.nkb - wc.k);
+        const int x = (wc.kb0 + wc.k) * (kPKB / 4);   // byte offset of the stage in the row
+        mbar_arrive_expect_tx(full(st), kPWStage + nsub * C::kActSub);
+        uint8_t* wdst = s_w + st * kPWStage;
+        tma_load_2d(smem_u32(wdst), wc.wmap, full(st), x, wc.r0, pol_w);
+        tma_load_2d(smem_u32(wdst + kPWStage / 2), wc.wmap, full(st), x, wc.r1, pol_w);
         ++wi;
-        if (++wc.k == wc.nkb) load_cur(wc, wc.ui + 1);
+        wc.k += kPSub;
+        if (wc.k >= wc.nkb) load_cur(wc, wc.ui + 1);
       }
-      // Abort path: stages whose weights were requested but whose activation tile was not
-      // get it now (the workspace buffer is valid memory), so that every started stage
+      // Abort path: stages whose weights were requested but whose activations were not get
+      // them now (the workspace buffer is valid memory), so that every started stage
       // completes; then wait until every copy this thread started has landed.
       while (ai < wi && ac.ui < u_end) {
-        const int s = static_cast<int>(ai % kPStages);
-        tma_load_2d(smem_u32(s_act + s * C::kAct), ac.amap, full(s), (ac.kb0 + ac.k) * kPKB, 0,
-                    pol_a);
+        const int st = static_cast<int>(ai % S);
+        const int nsub = min(kPSub, ac.nkb - ac.k);
+        for (int i = 0; i < nsub; ++i)
+          tma_load_2d(smem_u32(s_act + st * C::kAct + i * C::kActSub), ac.amap, full(st),
+                      (ac.kb0 + ac.k + i) * kPKB, 0, pol_a);
         ++ai;
-        if (++ac.k == ac.nkb) load_cur(ac, ac.ui + 1);
+        ac.k += kPSub;
+        if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
       }
-      for (int64_t i = wi > kPStages ? wi - kPStages : 0; i < wi; ++i)
-        mbar_wait_bounded(full(static_cast<int>(i % kPStages)),
-                          static_cast<uint32_t>((i / kPStages) & 1), kPDrainNs, nullptr, status);
+      for (int64_t i = wi > S ? wi - S : 0; i < wi; ++i)
+        mbar_wait_bounded(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1),
+                          kPDrainNs, nullptr, status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
-      const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
-      int s = 0;
-      uint32_t ph = 0;
-      bool ok = true;
-      int n = 0;
-      int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
-      for (int ui = u_begin; ui < u_end && ok; ++ui, ++n) {
-        const int nkb = next_nkb;
-        if (ui + 1 < u_end) next_nkb = units[ui + 1].nkb;   // overlaps this unit's MMAs
-        const int b = n & 1;
-        if (n >= 2 &&
-            !mbar_wait_bounded(accempty(b), static_cast<uint32_t>(((n >> 1) - 1) & 1), limit_ns,
-                               abort_flag, status))
+    // The whole warp runs the loop (waits and their outcomes are warp-uniform) and one elected
+    // lane issues each MMA and commit.
+    constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
+    const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
+    int64_t c = 0;                       // stage counter
+    bool ok = true;
+    int n = 0;
+    int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
+    for (int ui = u_begin; ui < u_end && ok; ++ui, ++n) {
+      const int nkb = next_nkb;
+      if (ui + 1 < u_end) next_nkb = units[ui + 1].nkb;   // overlaps this unit's MMAs
+      const int b = n & 1;
+      if (n >= 2) {
+        const bool w = mbar_wait_bounded(accempty(b), static_cast<uint32_t>(((n >> 1) - 1) & 1),
+                                         limit_ns, abort_flag, status);
+        if (!__all_sync(0xFFFFFFFFu, w)) break;
+      }
+      tc_fence_after();
+      // accumulator b spans TMEM columns [64b, 64b + 64).  With BN <= 32 it holds two partial
+      // sums, even sub-blocks at column 64b and odd ones at 64b + 32: consecutive MMAs into
+      // different accumulators keep the tensor pipe busier than a chain on one (the epilogue
+      // adds the two, exactly, in int32).
+      const uint32_t d = tmem + static_cast<uint32_t>(b * 64);
+      for (int k = 0; k < nkb; k += kPSub, ++c) {
+        const int nsub = min(kPSub, nkb - k);
+        const int st = static_cast<int>(c % S);
+        const int gi = static_cast<int>(c % kPGroups);
+        const bool w = mbar_wait_bounded(afull(gi), static_cast<uint32_t>((c / kPGroups) & 1),
+                                         limit_ns, abort_flag, status);
+        if (!__all_sync(0xFFFFFFFFu, w)) {
+          ok = false;
           break;
+        }
         tc_fence_after();
-        const uint32_t d = tmem + static_cast<uint32_t>(b * 64);
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait_bounded(afull(s), ph, limit_ns, abort_flag, status)) {
+        for (int i = 0; i < nsub; ++i) {
+          // descriptor start address is in 16-byte units: a sub-tile is kActSub bytes, a
+          // 32-deep k step is 32 bytes within the 128-byte swizzled rows
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>((st * C::kAct + i * C::kActSub) >> 4);
+          const uint32_t ad = tmem + kPACol0 + (gi * kPSub + i) * 32;
+          const int j = k + i;                       // sub-block index within the unit
+          const uint32_t dj = kSplitAcc<BN> ? d + static_cast<uint32_t>((j & 1) * 32) : d;
+          const uint32_t first = kSplitAcc<BN> ? (j < 2) : (j == 0);
+          tc_mma_i8_ts_warp(dj, ad, bd, idesc, first ? 0u : 1u);
+          tc_mma_i8_ts_warp(dj, ad + 8, bd + 2, idesc, 1u);
+          tc_mma_i8_ts_warp(dj, ad + 16, bd + 4, idesc, 1u);
+          tc_mma_i8_ts_warp(dj, ad + 24, bd + 6, idesc, 1u);
+        }
+        tc_commit_warp(empty(st));
+      }
+      if (ok) tc_commit_warp(accfull(b));
+    }
+    // Drain: nothing this warp issued may still be running when TMEM is freed.
+    tc_commit_warp(drainbar);
+    mbar_wait_bounded(drainbar, 0u, kPDrainNs, nullptr, status);
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ unpack
+    // Each lane owns one tile row (= TMEM lane): per stage it reads its row's 128-byte weight
+    // line once and unpacks its sub-blocks (32 bytes, 128 codes each) into TMEM slots.
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    int64_t c = 0;                       // stage counter
+    bool ok = true;
+    for (int ui = u_begin; ui < u_end && ok; ++ui) {
+      const int nkb = units[ui].nkb;
+      for (int k = 0; k < nkb; k += kPSub, ++c) {
+        const int nsub = min(kPSub, nkb - k);
+        const int st = static_cast<int>(c % S);
+        const int gi = static_cast<int>(c % kPGroups);
+        bool w = mbar_wait_bounded(full(st), static_cast<uint32_t>((c / S) & 1), limit_ns,
+                                   abort_flag, status);
+        if (!__all_sync(0xFFFFFFFFu, w)) {
+          ok = false;
+          break;
+        }
+        // 128-byte swizzle: 16-byte chunk c of row r sits at chunk position c ^ (r mod 8)
+        const uint8_t* wrow = s_w + st * kPWStage + r * kPWRow;
+        uint4 ch[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          ch[cc] = *reinterpret_cast<const uint4*>(wrow + ((cc ^ (r & 7)) << 4));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(st));
+        // slot group gi was last read by the MMAs of stage c - 3: their commit completed
+        // empty((c - 3) % S).  (That barrier cannot have moved a further phase on: it needs
+        // this warp's arrival for stage c - 3 + S first.)
+        if (c >= kPGroups) {
+          const int64_t cp = c - kPGroups;
+          w = mbar_wait_bounded(empty(static_cast<int>(cp % S)), static_cast<uint32_t>((cp / S) & 1),
+                                limit_ns, abort_flag, status);
+          if (!__all_sync(0xFFFFFFFFu, w)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kAct) >> 4);
-          const uint32_t ad = tmem + kPACol0 + s * 32;
-          tc_mma_i8_ts(d, ad, bd, idesc, kb > 0 ? 1u : 0u);
-          tc_mma_i8_ts(d, ad + 8, bd + 2, idesc, 1u);
-          tc_mma_i8_ts(d, ad + 16, bd + 4, idesc, 1u);
-          tc_mma_i8_ts(d, ad + 24, bd + 6, idesc, 1u);
-          tc_commit(empty(s));
-          if (++s == kPStages) {
-            s = 0;
-            ph ^= 1u;
+        }
+        // all sub-blocks of the stage are stored before one wait: the store latency is paid
+        // once per stage, not once per sub-block
+#pragma unroll
+        for (int i = 0; i < kPSub; ++i) {
+          if (i < nsub) {
+            uint32_t uu[32];
+            const uint4 lo = ch[2 * i], hi = ch[2 * i + 1];
+            unpack_word4(lo.x, uu + 0);
+            unpack_word4(lo.y, uu + 4);
+            unpack_word4(lo.z, uu + 8);
+            unpack_word4(lo.w, uu + 12);
+            unpack_word4(hi.x, uu + 16);
+            unpack_word4(hi.y, uu + 20);
+            unpack_word4(hi.z, uu + 24);
+            unpack_word4(hi.w, uu + 28);
+            tc_st_32x32b_x32(tmem + lane_addr + kPACol0 + (gi * kPSub + i) * 32, uu);
           }
         }
-        if (ok) tc_commit(accfull(b));
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull(gi));
       }
-      // Drain: nothing this thread issued may still be running when TMEM is freed.
-      tc_commit(drainbar);
-      mbar_wait_bounded(drainbar, 0u, kPDrainNs, nullptr, status);
     }
   } else {
-    // ------------------------------------------------------------------ quantise, unpack, epilogue
+    // ------------------------------------------------------------------ quantise + epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    const int et = threadIdx.x - 64;
+    const int et = threadIdx.x - kPEpiT0;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+    constexpr int CH = C::kCh;
     bool ok = true;
-    int s = 0;
-    uint32_t ph = 0;
     int n = 0;
     int ui = u_begin;
     for (int L = 0; L < H.n_levels; ++L) {
-      // 1. quantise a share of this level's input rows (one warp per row)
+      // 1. quantise a share of this level's input rows (the 128 threads take one row at a time)
       const int ib = H.in_begin[L], ie = H.in_begin[L + 1];
       const int rows = (ie - ib) * T;
-      for (int rho = blockIdx.x; rho < rows && ok; rho += nct)
-        quant_row(ins[ib + rho / T], rho % T, H.eps, et, s_red_d, s_red_f, s_red_i);
+      if (rows > nct) {   // more rows than CTAs: one row per warp, four at once
+        // first every row this warp will quantise is requested into L2 at once
+        if (lane == 0)
+          for (int rho = blockIdx.x * 4 + (et >> 5); rho < rows; rho += nct * 4) {
+            const PIn& in = ins[ib + rho / T];
+            const int rb = in.K * (in.xdt == kInF16 ? 2 : 4);
+            bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(in.x) + static_cast<int64_t>(rho % T) * rb,
+                             static_cast<uint32_t>(rb));
+          }
+        __syncwarp();
+        for (int rho = blockIdx.x * 4 + (et >> 5); rho < rows && ok; rho += nct * 4)
+          quant_row_warp(ins[ib + rho / T], rho % T, H.eps, lane);
+      } else {
+        for (int rho = blockIdx.x; rho < rows && ok; rho += nct)
+          quant_row(ins[ib + rho / T], rho % T, H.eps, et, s_red_d, s_red_f, s_red_i);
+      }
       fence_proxy_async_global();   // the codes are read by TMA (async proxy) in other CTAs
       named_bar_sync(1, kPEpi);
       if (et == 0) {
         grid_arrive(lvl + 2 * L);
         // gamma and the code sums of this level are read below (staged per unit): wait until
-        // every CTA has quantised its rows (the unpack would wait for this anyway, through the
-        // activation tiles the producer loads after the same barrier)
+        // every CTA has quantised its rows
         s_qflag = grid_wait(lvl + 2 * L, static_cast<unsigned>(nct), poison, limit_ns, status) ? 1 : 0;
         if (!s_qflag) *abort_flag = 1;
       }
       named_bar_sync(1, kPEpi);
       if (!s_qflag) ok = false;
       // 2. this CTA's units of level L
-      while (ui < u_end && projs[units[ui].proj].level == L) {
-        // plan records are copied into registers (output stores cannot alias them) and the
-        // per-token scale and code sum are staged before the unpack, so their L2 latency
-        // overlaps it
+      while (ok && ui < u_end && projs[units[ui].proj].level == L) {
+        // plan records are copied into registers (output stores cannot alias them); the
+        // per-token scale and code sum are staged while the accumulator is still being built
         const PUnit u = units[ui];
         const PProj pj = projs[u.proj];
         const PIn in = ins[pj.in];
@@ -573,91 +846,62 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
           tsc[et] = __fmul_rn(__fdiv_rn(__ldcg(in.gamma + et), 127.0f), __ldg(pj.beta));
           trs[et] = __ldcg(in.rowsum + et);
         }
-        for (int kb = 0; kb < u.nkb && ok; ++kb) {
-          const bool w = mbar_wait_bounded(full(s), ph, limit_ns, abort_flag, status);
-          if (!__all_sync(0xFFFFFFFFu, w)) {
-            ok = false;
-            break;
-          }
-          const uint8_t* wrow = s_w + s * kPWStage + r * kPWRow;
-          const int sw = (r >> 2) & 1;
-          const uint4 lo = *reinterpret_cast<const uint4*>(wrow + 16 * sw);
-          const uint4 hi = *reinterpret_cast<const uint4*>(wrow + 16 * (sw ^ 1));
-          __syncwarp();
-          if (lane == 0) mbar_arrive(empty(s));
-          uint32_t uu[32];
-          unpack_word4(lo.x, uu + 0);
-          unpack_word4(lo.y, uu + 4);
-          unpack_word4(lo.z, uu + 8);
-          unpack_word4(lo.w, uu + 12);
-          unpack_word4(hi.x, uu + 16);
-          unpack_word4(hi.y, uu + 20);
-          unpack_word4(hi.z, uu + 24);
-          unpack_word4(hi.w, uu + 28);
-          tc_st_32x32b_x32(tmem + lane_addr + kPACol0 + s * 32, uu);
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(afull(s));
-          if (++s == kPStages) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-        // epilogue of unit ui
         const int b = n & 1;
-        if (ok) {
-          const bool w = mbar_wait_bounded(accfull(b), static_cast<uint32_t>((n >> 1) & 1),
-                                           limit_ns, abort_flag, status);
-          ok = __all_sync(0xFFFFFFFFu, w);
-        }
-        ok = named_bar_and(1, kPEpi, ok);
+        const bool w = mbar_wait_bounded(accfull(b), static_cast<uint32_t>((n >> 1) & 1),
+                                         limit_ns, abort_flag, status);
+        ok = named_bar_and(1, kPEpi, __all_sync(0xFFFFFFFFu, w));   // also publishes tsc/trs
         if (!ok) break;
         tc_fence_after();
-        int32_t acc[BN];
-        {
-          uint32_t v[32];
-#pragma unroll
-          for (int c0 = 0; c0 < BN; c0 += (BN < 32 ? BN : 32)) {
-            if constexpr (BN < 32) {
-              tc_ld_32x32b_x16(tmem + lane_addr + static_cast<uint32_t>(b * 64 + c0), v);
-            } else {
-              tc_ld_32x32b_x32(tmem + lane_addr + static_cast<uint32_t>(b * 64 + c0), v);
-            }
-            tc_wait_ld();
-#pragma unroll
-            for (int j = 0; j < (BN < 32 ? BN : 32); ++j) acc[c0 + j] = static_cast<int32_t>(v[j]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(accempty(b));
-        named_bar_sync(1, kPEpi);   // tsc/trs written by other threads
+        const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(b * 64);
+        const bool two = kSplitAcc<BN> && u.nkb > 1;   // the odd-sub-block partial exists
         if (u.nsplit == 1) {
-          finalize_tile<BN>(pj, u.tile, T, acc, r, tsc, trs, xbuf, ostage);
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
+            int32_t v[CH];
+            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), two, v);
+            finalize_chunk<CH>(pj, u.tile, T, c0, v, r, tsc, trs, xbuf, ostage);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(accempty(b));
+          store_tile(pj, u.tile, T, et, ostage);
         } else {
           int32_t* mine = parts + static_cast<int64_t>(u.part_off + u.split) * BN * 128;
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
+            int32_t v[CH];
+            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), two, v);
 #pragma unroll
-          for (int j = 0; j < BN; ++j) __stcg(mine + j * 128 + r, acc[j]);
+            for (int jj = 0; jj < CH; ++jj) __stcg(mine + (c0 + jj) * 128 + r, v[jj]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(accempty(b));
           __threadfence();
           named_bar_sync(1, kPEpi);
           if (et == 0) s_flag = (atomicAdd(tilectr + u.tile_id, 1u) == static_cast<unsigned>(u.nsplit - 1));
           named_bar_sync(1, kPEpi);
           if (s_flag) {
             __threadfence();
-            // add the other splits in split order (int32: exact in any order)
-            for (int sp = 0; sp < u.nsplit; ++sp) {
-              if (sp == u.split) continue;
-              const int32_t* other = parts + static_cast<int64_t>(u.part_off + sp) * BN * 128;
+            // the last split to finish adds all partial sums in split order (int32: exact in
+            // any order) and finalises the tile
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
+              int32_t v[CH];
 #pragma unroll
-              for (int j = 0; j < BN; ++j) acc[j] += __ldcg(other + j * 128 + r);
+              for (int jj = 0; jj < CH; ++jj) v[jj] = 0;
+              for (int sp = 0; sp < u.nsplit; ++sp) {
+                const int32_t* src = parts + static_cast<int64_t>(u.part_off + sp) * BN * 128;
+#pragma unroll
+                for (int jj = 0; jj < CH; ++jj) v[jj] += __ldcg(src + (c0 + jj) * 128 + r);
+              }
+              finalize_chunk<CH>(pj, u.tile, T, c0, v, r, tsc, trs, xbuf, ostage);
             }
-            finalize_tile<BN>(pj, u.tile, T, acc, r, tsc, trs, xbuf, ostage);
+            store_tile(pj, u.tile, T, et, ostage);
             if (et == 0) tilectr[u.tile_id] = 0u;   // ready for the next run
           }
-          named_bar_sync(1, kPEpi);
         }
-        named_bar_sync(1, kPEpi);
+        named_bar_sync(1, kPEpi);   // ostage, tsc and trs are reused by the next unit
         ++n;
         ++ui;
       }
@@ -817,9 +1061,12 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
     std::vector<PUnit> lu;
     for (int i = 0; i < n; ++i) {
       if (p[i].level != L) continue;
+      // splits fall on stage boundaries (kPSub k-blocks), so that only the last stage of a
+      // row can be partial
       const int nkb = static_cast<int>(p[i].K / kPKB);
+      const int nst = (nkb + kPSub - 1) / kPSub;
       const int ns = static_cast<int>(std::min<int64_t>(
-          {static_cast<int64_t>(kMaxSplit), static_cast<int64_t>(nkb), (nkb + target - 1) / target}));
+          {static_cast<int64_t>(kMaxSplit), static_cast<int64_t>(nst), (nkb + target - 1) / target}));
       for (int t = 0; t < p[i].N / 128; ++t) {
         const int part_off = ns > 1 ? part_slots : 0;
         if (ns > 1) part_slots += ns;
@@ -827,8 +1074,8 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
           PUnit u;
           u.proj = i;
           u.tile = t;
-          u.kb0 = sp * nkb / ns;
-          u.nkb = (sp + 1) * nkb / ns - u.kb0;
+          u.kb0 = kPSub * (sp * nst / ns);
+          u.nkb = std::min(nkb, kPSub * ((sp + 1) * nst / ns)) - u.kb0;
           u.split = sp;
           u.nsplit = ns;
           u.tile_id = tile_base[i] + t;
@@ -917,13 +1164,13 @@ cudaError_t launch_program(const void* ws, int nct, unsigned* status, cudaStream
   cudaError_t ae = cudaSuccess;
   std::call_once(once[dev & 63], [&] {
     ae = cudaFuncSetAttribute(program_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              C::kSmem < 118 * 1024 ? 118 * 1024 : C::kSmem);
+                              C::kSmem);
   });
   if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(nct));
   cfg.blockDim = dim3(kPThreads);
-  cfg.dynamicSmemBytes = C::kSmem < 118 * 1024 ? 118 * 1024 : C::kSmem;
+  cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -957,13 +1204,14 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   st = build_plan(p, n, T, eps, reinterpret_cast<uintptr_t>(ws), nct, P);
   if (st != MMF_OK) return st;
   if (ws_bytes < P.bytes) return MMF_ERR_WORKSPACE;
-  // tensor maps: packed weights (box 64 rows x 32 B, 32-byte swizzle) and activation codes
-  // (box BN rows x 128 B, 128-byte swizzle), exactly as the single-projection kernel
+  // tensor maps: packed weights (box 64 rows x 128 B, 128-byte swizzle: one line of each row
+  // per stage; boxes reaching past the end of a row read zeros) and activation codes (box BN
+  // rows x 128 B, 128-byte swizzle)
   P.maps.resize(P.projs.size() + P.ins.size());
   for (size_t i = 0; i < P.projs.size(); ++i) {
     const PProj& q = P.projs[i];
     if (!make_tmap_2d_u8(&P.maps[i], q.Wp, static_cast<uint64_t>(q.K / 4), static_cast<uint64_t>(q.N),
-                         static_cast<uint64_t>(q.K / 4), kPWRow, 64, CU_TENSOR_MAP_SWIZZLE_32B))
+                         static_cast<uint64_t>(q.K / 4), kPWRow, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return MMF_ERR_CUDA;
   }
   for (size_t k = 0; k < P.ins.size(); ++k) {

@@ -237,33 +237,35 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
-      const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
-      int s = 0;
-      uint32_t ph = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait_bounded(afull(s), ph, p.wait_limit_ns, abort_flag, p.status)) break;
-        tc_fence_after();
-        // descriptor start address is in 16-byte units: a stage is kActStage bytes, a 32-deep
-        // k step is 32 bytes within the 128-byte swizzled rows
-        const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kActStage) >> 4);
-        const uint32_t ad = tmem + C::kACol0 + s * 32;
-        tc_mma_i8_ts(tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);   // kb counts this CTA's range
-        tc_mma_i8_ts(tmem, ad + 8, bd + 2, idesc, 1u);
-        tc_mma_i8_ts(tmem, ad + 16, bd + 4, idesc, 1u);
-        tc_mma_i8_ts(tmem, ad + 24, bd + 6, idesc, 1u);
-        tc_commit(empty(s));
-        if (++s == C::kStages) {
-          s = 0;
-          ph ^= 1u;
-        }
+    // The whole warp runs the loop (waits and their outcomes are warp-uniform) and one elected
+    // lane issues each MMA and commit.
+    constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
+    const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const bool w = mbar_wait_bounded(afull(s), ph, p.wait_limit_ns, abort_flag, p.status);
+      if (!__all_sync(0xFFFFFFFFu, w)) break;
+      tc_fence_after();
+      // descriptor start address is in 16-byte units: a stage is kActStage bytes, a 32-deep
+      // k step is 32 bytes within the 128-byte swizzled rows
+      const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kActStage) >> 4);
+      const uint32_t ad = tmem + C::kACol0 + s * 32;
+      tc_mma_i8_ts_warp(tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);   // kb counts this CTA's range
+      tc_mma_i8_ts_warp(tmem, ad + 8, bd + 2, idesc, 1u);
+      tc_mma_i8_ts_warp(tmem, ad + 16, bd + 4, idesc, 1u);
+      tc_mma_i8_ts_warp(tmem, ad + 24, bd + 6, idesc, 1u);
+      tc_commit_warp(empty(s));
+      if (++s == C::kStages) {
+        s = 0;
+        ph ^= 1u;
       }
-      // Signals the epilogue; in the abort path it also tells this thread when the MMAs it
-      // issued have finished, so TMEM is not freed under them.
-      tc_commit(accfull);
-      mbar_wait_bounded(accfull, 0, kDrainNs, nullptr, p.status);
     }
+    // Signals the epilogue; in the abort path it also tells this warp when the MMAs it issued
+    // have finished, so TMEM is not freed under them.
+    tc_commit_warp(accfull);
+    mbar_wait_bounded(accfull, 0, kDrainNs, nullptr, p.status);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ unpack + epilogue
     const int q = warp & 3;              // TMEM lane quarter this warp may access
