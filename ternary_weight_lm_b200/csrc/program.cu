@@ -56,7 +56,7 @@ constexpr int kPACol0 = 128;               // TMEM: accumulators at 0 and 64, sl
 constexpr int kMaxLevels = 128;
 constexpr int kMaxProj = 1024;
 constexpr int kMaxSplit = 16;
-constexpr int kMinSplitKb = 8;             // latency beats spreading at decode sizes
+constexpr int kMinSplitKb = 32;            // a split tile costs a few microseconds of reduction
 constexpr uint64_t kPDrainNs = 2000000000ull;
 static_assert(kPACol0 + kPSlots * 32 == 512, "TMEM columns");
 // Two partial accumulators per unit (even / odd sub-blocks) when they fit in the unit's 64
@@ -396,47 +396,54 @@ __device__ __forceinline__ void finalize_chunk(const PProj& pj, int tile, int T,
                                                const int32_t* __restrict__ trs,
                                                float* __restrict__ xbuf,
                                                __half* __restrict__ ostage) {
+  // every shared-memory operand is read into registers before the first store: the compiler
+  // cannot tell these buffers apart, and loads interleaved with stores would run one by one
+  float f[CH];
+  {
+    float sc[CH];
+    int32_t rs[CH];
+#pragma unroll
+    for (int jj = 0; jj < CH; ++jj) {
+      sc[jj] = tsc[c0 + jj];
+      rs[jj] = trs[c0 + jj];
+    }
+#pragma unroll
+    for (int jj = 0; jj < CH; ++jj) f[jj] = static_cast<float>(v[jj] - rs[jj]) * sc[jj];
+  }
   if (!pj.glu) {
     if (pj.ydt == MMF_F16) {
 #pragma unroll
-      for (int jj = 0; jj < CH; ++jj) {
-        const int j = c0 + jj;
-        if (j < T)
-          ostage[j * 128 + r] = __float2half_rn(static_cast<float>(v[jj] - trs[j]) * tsc[j]);
-      }
+      for (int jj = 0; jj < CH; ++jj)
+        if (c0 + jj < T) ostage[(c0 + jj) * 128 + r] = __float2half_rn(f[jj]);
     } else {
-      const int64_t n = static_cast<int64_t>(tile) * 128 + r;
+      float* y = reinterpret_cast<float*>(pj.y) + static_cast<int64_t>(tile) * 128 + r;
 #pragma unroll
-      for (int jj = 0; jj < CH; ++jj) {
-        const int j = c0 + jj;
-        if (j < T)
-          reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * pj.N + n] =
-              static_cast<float>(v[jj] - trs[j]) * tsc[j];
-      }
+      for (int jj = 0; jj < CH; ++jj)
+        if (c0 + jj < T) y[static_cast<int64_t>(c0 + jj) * pj.N] = f[jj];
     }
     return;
   }
   if (r >= 64) {
 #pragma unroll
-    for (int jj = 0; jj < CH; ++jj) {
-      const int j = c0 + jj;
-      xbuf[jj * 64 + (r - 64)] = j < T ? static_cast<float>(v[jj] - trs[j]) * tsc[j] : 0.0f;
-    }
+    for (int jj = 0; jj < CH; ++jj) xbuf[jj * 64 + (r - 64)] = f[jj];
   }
   named_bar_sync(1, kPEpi);
   if (r < 64) {
-    const int64_t I = pj.N / 2;
+    float u[CH];
 #pragma unroll
-    for (int jj = 0; jj < CH; ++jj) {
-      const int j = c0 + jj;
-      if (j < T) {
-        const float g = static_cast<float>(v[jj] - trs[j]) * tsc[j];
-        const float h = __fdividef(g, 1.0f + expf(-g)) * xbuf[jj * 64 + r];
-        if (pj.ydt == MMF_F16)
-          ostage[j * 64 + r] = __float2half_rn(h);
-        else
-          reinterpret_cast<float*>(pj.y)[static_cast<int64_t>(j) * I + static_cast<int64_t>(tile) * 64 + r] = h;
-      }
+    for (int jj = 0; jj < CH; ++jj) u[jj] = xbuf[jj * 64 + r];
+#pragma unroll
+    for (int jj = 0; jj < CH; ++jj) f[jj] = __fdividef(f[jj], 1.0f + expf(-f[jj])) * u[jj];
+    if (pj.ydt == MMF_F16) {
+#pragma unroll
+      for (int jj = 0; jj < CH; ++jj)
+        if (c0 + jj < T) ostage[(c0 + jj) * 64 + r] = __float2half_rn(f[jj]);
+    } else {
+      float* y = reinterpret_cast<float*>(pj.y) + static_cast<int64_t>(tile) * 64 + r;
+      const int64_t I = pj.N / 2;
+#pragma unroll
+      for (int jj = 0; jj < CH; ++jj)
+        if (c0 + jj < T) y[static_cast<int64_t>(c0 + jj) * I] = f[jj];
     }
   }
   named_bar_sync(1, kPEpi);   // xbuf is reused by the next chunk
@@ -845,6 +852,9 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         if (et < T) {
           tsc[et] = __fmul_rn(__fdiv_rn(__ldcg(in.gamma + et), 127.0f), __ldg(pj.beta));
           trs[et] = __ldcg(in.rowsum + et);
+        } else if (et < 64) {
+          tsc[et] = 0.0f;   // padding tokens of the last chunk
+          trs[et] = 0;
         }
         const int b = n & 1;
         const bool w = mbar_wait_bounded(accfull(b), static_cast<uint32_t>((n >> 1) & 1),
@@ -866,13 +876,17 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
           if (lane == 0) mbar_arrive(accempty(b));
           store_tile(pj, u.tile, T, et, ostage);
         } else {
-          int32_t* mine = parts + static_cast<int64_t>(u.part_off + u.split) * BN * 128;
+          // every split adds its partial sums into the tile's int32 accumulator in the
+          // workspace (fire-and-forget reductions; integer addition is exact in any order);
+          // the split that finishes last reads the total once, finalises the tile and zeroes
+          // the accumulator for the next run
+          int32_t* tacc = parts + static_cast<int64_t>(u.part_off) * BN * 128;
 #pragma unroll 1
           for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
             int32_t v[CH];
             load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), two, v);
 #pragma unroll
-            for (int jj = 0; jj < CH; ++jj) __stcg(mine + (c0 + jj) * 128 + r, v[jj]);
+            for (int jj = 0; jj < CH; ++jj) atomicAdd(tacc + (c0 + jj) * 128 + r, v[jj]);
           }
           tc_fence_before();
           __syncwarp();
@@ -883,18 +897,13 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
           named_bar_sync(1, kPEpi);
           if (s_flag) {
             __threadfence();
-            // the last split to finish adds all partial sums in split order (int32: exact in
-            // any order) and finalises the tile
 #pragma unroll 1
             for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
               int32_t v[CH];
 #pragma unroll
-              for (int jj = 0; jj < CH; ++jj) v[jj] = 0;
-              for (int sp = 0; sp < u.nsplit; ++sp) {
-                const int32_t* src = parts + static_cast<int64_t>(u.part_off + sp) * BN * 128;
+              for (int jj = 0; jj < CH; ++jj) v[jj] = __ldcg(tacc + (c0 + jj) * 128 + r);
 #pragma unroll
-                for (int jj = 0; jj < CH; ++jj) v[jj] += __ldcg(src + (c0 + jj) * 128 + r);
-              }
+              for (int jj = 0; jj < CH; ++jj) __stcg(tacc + (c0 + jj) * 128 + r, 0);
               finalize_chunk<CH>(pj, u.tile, T, c0, v, r, tsc, trs, xbuf, ostage);
             }
             store_tile(pj, u.tile, T, et, ostage);
@@ -1068,8 +1077,8 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
       const int ns = static_cast<int>(std::min<int64_t>(
           {static_cast<int64_t>(kMaxSplit), static_cast<int64_t>(nst), (nkb + target - 1) / target}));
       for (int t = 0; t < p[i].N / 128; ++t) {
-        const int part_off = ns > 1 ? part_slots : 0;
-        if (ns > 1) part_slots += ns;
+        const int part_off = ns > 1 ? part_slots : 0;   // one int32 accumulator tile per split tile
+        if (ns > 1) part_slots += 1;
         for (int sp = 0; sp < ns; ++sp) {
           PUnit u;
           u.proj = i;
@@ -1233,6 +1242,11 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // pageable source: the copy has consumed the host buffer when cudaMemcpyAsync returns
   if (cudaMemcpyAsync(ws, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MMF_ERR_CUDA;
+  // split tiles accumulate into zeroed int32 tiles (each run leaves them zeroed again)
+  if (P.bytes > static_cast<size_t>(P.h.off_part) &&
+      cudaMemsetAsync(static_cast<uint8_t*>(ws) + P.h.off_part, 0,
+                      P.bytes - static_cast<size_t>(P.h.off_part), s) != cudaSuccess)
     return MMF_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lk(g_runs_mu);
