@@ -40,26 +40,32 @@ constexpr int kEpiThreads = 128;
 constexpr uint64_t kDrainNs = 2000000000ull;
 constexpr int64_t kSplitTargetCtas = 148;       // SMs of a B200
 
-template <int BN>
+// TC: TMEM columns a CTA allocates.  512: one CTA owns the SM.  256: two CTAs share an SM
+// (half the shared memory each), so one CTA's epilogue overlaps the other's main loop.
+template <int BN, int TC = 512>
 struct Cfg {
   static constexpr int kActStage = BN * kKB;               // int8 activation tile
   static constexpr int kStage = kActStage + kWStageBytes;
   // One ring: stage s of shared memory and slot s of TMEM (the unpacked weights of that
   // stage) are filled and freed together, so every role waits on one barrier per k-block.
-  static constexpr int kTmemCols = 512;                    // one CTA per SM owns all of TMEM
+  static constexpr int kTmemCols = TC;
   static constexpr int kACol0 = ((BN + 31) / 32) * 32;     // first TMEM column of A slots
   static constexpr int kSlotsMax = (kTmemCols - kACol0) / 32;
-  static constexpr int kStagesSmem = (214 * 1024) / kStage;
+  static constexpr int kSmemBudget = TC == 512 ? 214 * 1024 : 108 * 1024;
+  static constexpr int kStagesSmem = kSmemBudget / kStage;
   static constexpr int kS0 = kStagesSmem < kSlotsMax ? kStagesSmem : kSlotsMax;
   static constexpr int kStages = kS0 > 16 ? 16 : kS0;
   static constexpr int kChunk = BN < 32 ? BN : 32;         // epilogue token columns per pass
   static constexpr int kBarBytes = 8 * (3 * kStages + 1);
   static constexpr int kTokBytes = 8 * BN;                 // per-token scale and code sum
   static constexpr int kSmemUsed = 1024 + kStages * kStage + kBarBytes + kTokBytes;
-  // At least ~116 KB so only one CTA lives on an SM (its TMEM allocation never waits).
-  static constexpr int kSmem = kSmemUsed < 118 * 1024 ? 118 * 1024 : kSmemUsed;
+  // TC == 512: at least ~116 KB, so only one CTA lives on an SM (its TMEM allocation never
+  // waits).  TC == 256: at most ~112 KB, so exactly two fit, and their TMEM halves fit too.
+  static constexpr int kSmem =
+      TC == 512 ? (kSmemUsed < 118 * 1024 ? 118 * 1024 : kSmemUsed) : kSmemUsed;
   static_assert(kStages >= 4, "pipeline needs four stages");
   static_assert(kSmem <= 227 * 1024, "shared memory per block");
+  static_assert(TC == 512 || kSmem <= 112 * 1024, "two CTAs per SM");
   static_assert(kChunk * 128 * 4 <= kStages * kActStage, "epilogue staging must fit");
 };
 
@@ -95,7 +101,7 @@ __device__ __forceinline__ float sigmoid_mul(float g, float u) {
 // adding the C partial sums (exact int32) read from each CTA's shared memory.  Thread et is
 // tile row et (non-GLU) or output column et < 64 (GLU: row et is the gated half, row et + 64
 // the multiplier).
-template <int BN>
+template <int BN, int TC>
 __device__ __forceinline__ void split_k_reduce(const Params& p, int csize, int64_t t0, int r0,
                                                const uint8_t* s_act, const float* s_scale,
                                                const int32_t* s_rsum) {
@@ -139,11 +145,11 @@ __device__ __forceinline__ void split_k_reduce(const Params& p, int csize, int64
   }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int TC>
+__global__ void __launch_bounds__(kThreads, TC == 512 ? 1 : 2)
 ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                     const Params p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, TC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -432,7 +438,7 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   if (csize > 1) {
     // Every thread of every CTA of the cluster reaches both barriers on every path.
     cluster_sync_all();
-    if (warp >= 2) split_k_reduce<BN>(p, csize, t0, r0, s_act, s_scale, s_rsum);
+    if (warp >= 2) split_k_reduce<BN, TC>(p, csize, t0, r0, s_act, s_scale, s_rsum);
     cluster_sync_all();   // peers' partial sums stay readable until everyone is done
   }
   if (warp == 1) {
@@ -442,16 +448,16 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   }
 }
 
-template <int BN>
+template <int BN, int TC = 512>
 cudaError_t launch_bn(const GemmCall& c, cudaStream_t s) {
-  using Cf = Cfg<BN>;
+  using Cf = Cfg<BN, TC>;
   static std::once_flag attr_once[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   cudaError_t attr_err = cudaSuccess;
   std::call_once(attr_once[dev & 63], [&] {
-    attr_err = cudaFuncSetAttribute(ternary_gemm_kernel<BN>,
+    attr_err = cudaFuncSetAttribute(ternary_gemm_kernel<BN, TC>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmem);
   });
   if (attr_err != cudaSuccess) return attr_err;
@@ -506,7 +512,7 @@ cudaError_t launch_bn(const GemmCall& c, cudaStream_t s) {
   attrs[1].val.clusterDim.z = static_cast<unsigned>(csize);
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, ternary_gemm_kernel<BN>, tm_w, tm_a, p);
+  return cudaLaunchKernelEx(&cfg, ternary_gemm_kernel<BN, TC>, tm_w, tm_a, p);
 }
 
 }  // namespace
@@ -516,7 +522,9 @@ cudaError_t launch_ternary_gemm(const GemmCall& c, cudaStream_t s) {
   if (c.T <= 32) return launch_bn<32>(c, s);
   if (c.T <= 64) return launch_bn<64>(c, s);
   if (c.T <= 128) return launch_bn<128>(c, s);
-  return launch_bn<256>(c, s);
+  // prefill: 128-token tiles, two CTAs per SM, so that one CTA's epilogue overlaps the
+  // other's main loop
+  return launch_bn<128, 256>(c, s);
 }
 
 namespace {
