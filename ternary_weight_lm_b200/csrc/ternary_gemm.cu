@@ -218,8 +218,13 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();   // weights: each byte is used once
-      const uint64_t pol_a = l2_policy_evict_last();    // activations: reused by every tile
+      // One token tile (decode): each weight byte is used once, the activation tile by every
+      // CTA.  Several token tiles (prefill): every token tile re-reads the whole weight
+      // matrix, so the weights stay in L2; an activation tile is read by the row tiles that run
+      // at about the same time.
+      const bool many_tok = gridDim.y > 1;
+      const uint64_t pol_w = many_tok ? l2_policy_evict_last() : l2_policy_evict_first();
+      const uint64_t pol_a = many_tok ? l2_policy_evict_normal() : l2_policy_evict_last();
       int issued = 0;
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % C::kStages;
