@@ -156,16 +156,20 @@ typedef struct {
   mmf_dtype ydt;
 } mmf_projection;
 
-/* Workspace bytes a program of n projections at T tokens needs (plan, quantised inputs,
- * split-K partial sums and counters).  0 if the program is not supported (T > 64, more than
- * 1024 projections or 128 levels, or a shape outside the limits). */
+/* Workspace bytes a program of n projections at T tokens needs: the plan, the quantised
+ * inputs, split-K accumulators and counters, and a re-tiled copy of every projection's packed
+ * weights (N*K/4 bytes each, rounded up to whole 512-wide k-stages).  0 if the program is not
+ * supported (T > 64, more than 1024 projections or 128 levels, or a shape outside the limits). */
 size_t mmf_program_workspace_bytes(const mmf_projection* p, int n, int64_t T);
 
 /* Plans a program into `ws` ([P1], [P3]; [P4] figure items 4 and 5, for every projection):
  * groups projections that share an input into one quantisation, splits every level's
- * k-blocks evenly over the SMs, encodes the tensor maps and zeroes the counters.  The
- * pointers in `p` are baked into the plan: every later mmf_program_run reads and writes those
- * same buffers.  Copies the plan with stream-ordered copies on `stream`.  1 <= T <= 64. */
+ * k-blocks over the SMs and zeroes the counters.  It also re-tiles every projection's packed
+ * weights (Wp, canonical layout L1) into the workspace, in blocks that one contiguous copy
+ * brings on chip: runs read that copy, so Wp may be freed after the init has executed, and a
+ * change of the weights needs a new init.  The other pointers in `p` are baked into the plan:
+ * every later mmf_program_run reads and writes those same buffers.  All work is
+ * stream-ordered on `stream`.  1 <= T <= 64. */
 mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T, float eps, void* ws,
                             size_t ws_bytes, void* stream);
 

@@ -12,14 +12,15 @@
 // costs microseconds of latency.  Here one CTA per SM runs the whole program:
 //   for each dependency level L
 //     1. the four epilogue warps of every CTA quantise a share of the level's input rows
-//        (RMSNorm + per-token absmax int8, one warp per row), then arrive on grid barrier Q[L];
+//        (RMSNorm + per-token absmax int8), then arrive on grid barrier Q[L];
 //     2. each CTA runs its planned units (a 128-row weight tile and a range of k-blocks): a
-//        TMA producer streams packed weights (ahead of time, across levels: weights do not
-//        depend on activations) and, once Q[L] has passed, the activation codes; four warps
-//        unpack the 2-bit codes into TMEM; one thread issues tcgen05 kind::i8 MMAs into one of
-//        two TMEM accumulators; the epilogue dequantises (and applies the GLU) or, for a tile
-//        split over several CTAs, hands its int32 partial sum to whichever CTA finishes the
-//        tile last, which adds the partials in split order (exact) and finalises the tile;
+//        producer thread streams the unit's packed weights (re-tiled at init into 16 KB
+//        blocks, one contiguous bulk copy per stage; ahead of time, across levels) and, once
+//        Q[L] has passed, the stage's activation codes (written tiled by step 1, one copy);
+//        four warps unpack the 2-bit codes into TMEM; a fifth issues tcgen05 kind::i8 MMAs into
+//        one of two TMEM accumulators; four more dequantise (and apply the GLU) or, for a tile
+//        split over several CTAs, add the int32 partial sums into the tile's accumulator, the
+//        last split finishing the tile;
 //     3. every CTA arrives on grid barrier O[L]; the next level may read this level's outputs.
 // Grid barriers are counters in the workspace with bounded waits; a timeout anywhere sets a
 // poison flag that makes every other wait give up too, and is reported as MMF_ERR_TIMEOUT.
@@ -64,20 +65,29 @@ static_assert(kPACol0 + kPSlots * 32 == 512, "TMEM columns");
 template <int BN>
 constexpr bool kSplitAcc = BN <= 32;
 
+// nst: stages of K = 512 per row (the last one may be partial).  Wt: the projection's packed
+// weights re-tiled in the workspace, [tile][stage][128 rows x 128 B], each 16 KB block stored as
+// the shared-memory image the unpack warps read (128-byte swizzle: 16-byte chunk c of row r at
+// position c ^ (r mod 8)); bytes past the end of a row are zero.
 struct PProj {
   const uint8_t* Wp;
+  const uint8_t* Wt;
   const float* beta;
   void* y;
-  int32_t K, N, glu, ydt, in, level, wmap, pad;
+  int32_t K, N, glu, ydt, in, level, nst, pad;
 };
 
+// A: the input's int8 codes, tiled as [stage][sub-block][BN token rows][128 B] with the same
+// 128-byte swizzle (chunk c of token row t at position c ^ (t mod 8)), so that the activation
+// sub-tiles of a stage are one contiguous block in the layout the MMA reads.  Token rows T..BN-1
+// are never written: they only feed accumulator columns that are not stored.
 struct PIn {
   const void* x;
   const float* g;
   int8_t* A;
   float* gamma;
   int32_t* rowsum;
-  int32_t K, xdt, level, amap;
+  int32_t K, xdt, level, nst;
 };
 
 struct PUnit {
@@ -88,7 +98,7 @@ struct PHeader {
   int32_t n_proj, n_in, n_levels, n_ctas, n_units, T, BN, n_tiles;
   float eps;
   int32_t pad[3];
-  int64_t off_in, off_proj, off_units, off_ctaoff, off_maps, off_tilectr, off_levelctr, off_part;
+  int64_t off_in, off_proj, off_units, off_ctaoff, off_wt, off_tilectr, off_levelctr, off_part;
   int32_t in_begin[kMaxLevels + 1];
 };
 
@@ -147,6 +157,13 @@ __device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, 
   }
 }
 
+// Byte offset of code k of token t in an input's tiled codes (k a multiple of 4).
+__device__ __forceinline__ int64_t a_tiled(int t, int k, int bn) {
+  const int sub = k >> 7;                       // global sub-block index = 4 * stage + i
+  const int c = (k >> 4) & 7;
+  return (static_cast<int64_t>(sub) * bn + t) * 128 + ((c ^ (t & 7)) << 4) + (k & 15);
+}
+
 __device__ __forceinline__ void widen16(const uint4& a, int xdt, float (&v)[8], int& n) {
   if (xdt == kInF16) {
     const __half2* h = reinterpret_cast<const __half2*>(&a);
@@ -170,8 +187,8 @@ __device__ __forceinline__ void widen16(const uint4& a, int xdt, float (&v)[8], 
 // q = rne(xhat * (127/gamma))).  The row is read once (ld.global.cg: this launch may have
 // written it) into registers, at most 8 vectors of 16 bytes per thread (K <= 8192 fp16 /
 // 4096 fp32).  red_d/red_f/red_i: per-warp partials in shared memory.
-__device__ void quant_row(const PIn in, int t, float eps, int et, double* red_d, float* red_f,
-                          int* red_i) {
+__device__ void quant_row(const PIn in, int t, float eps, int et, int bn, double* red_d,
+                          float* red_f, int* red_i) {
   constexpr int kVmax = 8;
   const int K = in.K;
   const int E = in.xdt == kInF16 ? 8 : 4;
@@ -227,7 +244,6 @@ __device__ void quant_row(const PIn in, int t, float eps, int et, double* red_d,
   const float gm = fmaxf(amax, 1e-5f);
   const float s = __fdiv_rn(127.0f, gm);
   int rs = 0;
-  int8_t* ar = in.A + static_cast<int64_t>(t) * K;
 #pragma unroll
   for (int i = 0; i < kVmax; ++i) {
     const int vi = et + kPEpi * i;
@@ -245,9 +261,9 @@ __device__ void quant_row(const PIn in, int t, float eps, int et, double* red_d,
         wd[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (e & 3));
       }
       if (E == 8)
-        *reinterpret_cast<uint2*>(ar + vi * 8) = make_uint2(wd[0], wd[1]);
+        *reinterpret_cast<uint2*>(in.A + a_tiled(t, vi * 8, bn)) = make_uint2(wd[0], wd[1]);
       else
-        *reinterpret_cast<uint32_t*>(ar + vi * 4) = wd[0];
+        *reinterpret_cast<uint32_t*>(in.A + a_tiled(t, vi * 4, bn)) = wd[0];
     }
   }
 #pragma unroll
@@ -273,7 +289,7 @@ __device__ void quant_row(const PIn in, int t, float eps, int et, double* red_d,
 // Without a norm weight gamma = (max|x|)*inv exactly: rounding is monotone, so the largest
 // |x*inv| comes from the largest |x| (and *1.0f is exact).
 constexpr int kQW = 2;
-__device__ void quant_row_warp(const PIn in, int t, float eps, int lane) {
+__device__ void quant_row_warp(const PIn in, int t, float eps, int lane, int bn) {
   const int K = in.K;
   const int E = in.xdt == kInF16 ? 8 : 4;
   const int nvec = K / E;
@@ -337,7 +353,6 @@ __device__ void quant_row_warp(const PIn in, int t, float eps, int lane) {
   const float gm = fmaxf(amax, 1e-5f);
   const float s = __fdiv_rn(127.0f, gm);
   int rs = 0;
-  int8_t* ar = in.A + static_cast<int64_t>(t) * K;
 #pragma unroll 1
   for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
     uint4 raw[kQW];
@@ -363,9 +378,9 @@ __device__ void quant_row_warp(const PIn in, int t, float eps, int lane) {
           wd[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (e & 3));
         }
         if (E == 8)
-          *reinterpret_cast<uint2*>(ar + vi * 8) = make_uint2(wd[0], wd[1]);
+          *reinterpret_cast<uint2*>(in.A + a_tiled(t, vi * 8, bn)) = make_uint2(wd[0], wd[1]);
         else
-          *reinterpret_cast<uint32_t*>(ar + vi * 4) = wd[0];
+          *reinterpret_cast<uint32_t*>(in.A + a_tiled(t, vi * 4, bn)) = wd[0];
       }
     }
   }
@@ -568,7 +583,6 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   const PProj* projs = reinterpret_cast<const PProj*>(ws + H.off_proj);
   const PUnit* units = reinterpret_cast<const PUnit*>(ws + H.off_units);
   const int32_t* ctaoff = reinterpret_cast<const int32_t*>(ws + H.off_ctaoff);
-  const CUtensorMap* maps = reinterpret_cast<const CUtensorMap*>(ws + H.off_maps);
   unsigned* tilectr = reinterpret_cast<unsigned*>(const_cast<uint8_t*>(ws) + H.off_tilectr);
   unsigned* lvl = reinterpret_cast<unsigned*>(const_cast<uint8_t*>(ws) + H.off_levelctr);
   unsigned* poison = lvl + 2 * kMaxLevels;
@@ -581,19 +595,20 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    // A stage is up to four k-blocks of one unit: one 128-byte line of each of the tile's 128
-    // packed weight rows (two boxes of 64 rows) and one activation sub-tile per k-block.  The
-    // weights run ahead of the activations (they do not depend on them), up to a full ring.
+    // A stage is up to four k-blocks of one unit: the unit's 16 KB block of re-tiled weights
+    // (one 128-byte line of each of the tile's 128 rows) and the stage's activation sub-tiles,
+    // each one contiguous bulk copy.  The weights run ahead of the activations (they do not
+    // depend on them), up to a full ring.
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_a = l2_policy_evict_last();
-      // The unit records are read from the workspace once per unit into registers (the TMA
+      // The unit records are read from the workspace once per unit into registers (the copy
       // asm statements clobber memory, so a record read inside the stage loop would be
       // re-fetched from L2 for every stage).
       struct Cur {
-        int ui, k, nkb, kb0, r0, r1, level;
-        const CUtensorMap* wmap;
-        const CUtensorMap* amap;
+        int ui, k, nkb, kb0, level;
+        const uint8_t* w;     // this unit's first weight block
+        const int8_t* a;      // the input's tiled codes
       };
       auto load_cur = [&](Cur& c, int ui) {
         c.ui = ui;
@@ -604,15 +619,8 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         c.nkb = u.nkb;
         c.kb0 = u.kb0;
         c.level = pj.level;
-        if (pj.glu) {
-          c.r0 = u.tile * 64;
-          c.r1 = pj.N / 2 + u.tile * 64;
-        } else {
-          c.r0 = u.tile * 128;
-          c.r1 = c.r0 + 64;
-        }
-        c.wmap = maps + pj.wmap;
-        c.amap = maps + ins[pj.in].amap;
+        c.w = pj.Wt + (static_cast<int64_t>(u.tile) * pj.nst + u.kb0 / kPSub) * kPWStage;
+        c.a = ins[pj.in].A;
       };
       Cur wc, ac;
       load_cur(wc, u_begin);
@@ -620,6 +628,16 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       int64_t wi = 0, ai = 0;
       int q_level = -1;
       bool ok = true;
+      auto issue_act = [&]() {
+        const int st = static_cast<int>(ai % S);
+        const int nsub = min(kPSub, ac.nkb - ac.k);
+        // sub-blocks (kb0 + k) .. +nsub of the input, contiguous in its tiled codes
+        bulk_load(smem_u32(s_act + st * C::kAct), ac.a + static_cast<int64_t>(ac.kb0 + ac.k) * C::kActSub,
+                  static_cast<uint32_t>(nsub * C::kActSub), full(st), pol_a);
+        ++ai;
+        ac.k += kPSub;
+        if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
+      };
       while (ok && ac.ui < u_end) {
         // 1. the activation sub-tiles of every stage whose weights are already requested; at a
         //    new level, first wait until its codes exist
@@ -634,14 +652,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
             fence_proxy_async_global();
             q_level = ac.level;
           }
-          const int st = static_cast<int>(ai % S);
-          const int nsub = min(kPSub, ac.nkb - ac.k);
-          for (int i = 0; i < nsub; ++i)
-            tma_load_2d(smem_u32(s_act + st * C::kAct + i * C::kActSub), ac.amap, full(st),
-                        (ac.kb0 + ac.k + i) * kPKB, 0, pol_a);
-          ++ai;
-          ac.k += kPSub;
-          if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
+          issue_act();
         }
         if (!ok || wc.ui >= u_end) continue;
         // 2. the packed weights of the next stage
@@ -653,11 +664,9 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
           break;
         }
         const int nsub = min(kPSub, wc.nkb - wc.k);
-        const int x = (wc.kb0 + wc.k) * (kPKB / 4);   // byte offset of the stage in the row
         mbar_arrive_expect_tx(full(st), kPWStage + nsub * C::kActSub);
-        uint8_t* wdst = s_w + st * kPWStage;
-        tma_load_2d(smem_u32(wdst), wc.wmap, full(st), x, wc.r0, pol_w);
-        tma_load_2d(smem_u32(wdst + kPWStage / 2), wc.wmap, full(st), x, wc.r1, pol_w);
+        bulk_load(smem_u32(s_w + st * kPWStage), wc.w + static_cast<int64_t>(wc.k / kPSub) * kPWStage,
+                  kPWStage, full(st), pol_w);
         ++wi;
         wc.k += kPSub;
         if (wc.k >= wc.nkb) load_cur(wc, wc.ui + 1);
@@ -665,16 +674,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       // Abort path: stages whose weights were requested but whose activations were not get
       // them now (the workspace buffer is valid memory), so that every started stage
       // completes; then wait until every copy this thread started has landed.
-      while (ai < wi && ac.ui < u_end) {
-        const int st = static_cast<int>(ai % S);
-        const int nsub = min(kPSub, ac.nkb - ac.k);
-        for (int i = 0; i < nsub; ++i)
-          tma_load_2d(smem_u32(s_act + st * C::kAct + i * C::kActSub), ac.amap, full(st),
-                      (ac.kb0 + ac.k + i) * kPKB, 0, pol_a);
-        ++ai;
-        ac.k += kPSub;
-        if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
-      }
+      while (ai < wi && ac.ui < u_end) issue_act();
       for (int64_t i = wi > S ? wi - S : 0; i < wi; ++i)
         mbar_wait_bounded(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1),
                           kPDrainNs, nullptr, status);
@@ -715,18 +715,28 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
           break;
         }
         tc_fence_after();
-        for (int i = 0; i < nsub; ++i) {
-          // descriptor start address is in 16-byte units: a sub-tile is kActSub bytes, a
-          // 32-deep k step is 32 bytes within the 128-byte swizzled rows
-          const uint64_t bd = bdesc0 + static_cast<uint64_t>((st * C::kAct + i * C::kActSub) >> 4);
-          const uint32_t ad = tmem + kPACol0 + (gi * kPSub + i) * 32;
+        // descriptor start address is in 16-byte units: a sub-tile is kActSub bytes, a 32-deep
+        // k step is 32 bytes within the 128-byte swizzled rows
+        const uint64_t bst = bdesc0 + static_cast<uint64_t>((st * C::kAct) >> 4);
+        const uint32_t ast = tmem + kPACol0 + gi * kPSub * 32;
+        auto sub = [&](int i) {
+          const uint64_t bd = bst + static_cast<uint64_t>((i * C::kActSub) >> 4);
+          const uint32_t ad = ast + i * 32;
           const int j = k + i;                       // sub-block index within the unit
           const uint32_t dj = kSplitAcc<BN> ? d + static_cast<uint32_t>((j & 1) * 32) : d;
-          const uint32_t first = kSplitAcc<BN> ? (j < 2) : (j == 0);
+          const bool first = kSplitAcc<BN> ? (j < 2) : (j == 0);
           tc_mma_i8_ts_warp(dj, ad, bd, idesc, first ? 0u : 1u);
           tc_mma_i8_ts_warp(dj, ad + 8, bd + 2, idesc, 1u);
           tc_mma_i8_ts_warp(dj, ad + 16, bd + 4, idesc, 1u);
           tc_mma_i8_ts_warp(dj, ad + 24, bd + 6, idesc, 1u);
+        };
+        if (nsub == kPSub) {
+          // a full stage as straight-line code: a runtime loop here costs the tensor pipe
+          // about 40 % of its issue rate
+#pragma unroll
+          for (int i = 0; i < kPSub; ++i) sub(i);
+        } else {
+          for (int i = 0; i < nsub; ++i) sub(i);
         }
         tc_commit_warp(empty(st));
       }
@@ -751,8 +761,14 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         const int nsub = min(kPSub, nkb - k);
         const int st = static_cast<int>(c % S);
         const int gi = static_cast<int>(c % kPGroups);
-        bool w = mbar_wait_bounded(full(st), static_cast<uint32_t>((c / S) & 1), limit_ns,
-                                   abort_flag, status);
+        // Both conditions of this stage (its data landed; its slot group is free, see below)
+        // are tested in one statement first; the bounded waits run only if one is not met.
+        const int64_t cp = c - kPGroups;
+        const bool both = cp >= 0 && mbar_try_wait2(full(st), static_cast<uint32_t>((c / S) & 1),
+                                                     empty(static_cast<int>(cp % S)),
+                                                     static_cast<uint32_t>((cp / S) & 1));
+        bool w = both || mbar_wait_bounded(full(st), static_cast<uint32_t>((c / S) & 1),
+                                           limit_ns, abort_flag, status);
         if (!__all_sync(0xFFFFFFFFu, w)) {
           ok = false;
           break;
@@ -768,8 +784,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         // slot group gi was last read by the MMAs of stage c - 3: their commit completed
         // empty((c - 3) % S).  (That barrier cannot have moved a further phase on: it needs
         // this warp's arrival for stage c - 3 + S first.)
-        if (c >= kPGroups) {
-          const int64_t cp = c - kPGroups;
+        if (cp >= 0 && !both) {
           w = mbar_wait_bounded(empty(static_cast<int>(cp % S)), static_cast<uint32_t>((cp / S) & 1),
                                 limit_ns, abort_flag, status);
           if (!__all_sync(0xFFFFFFFFu, w)) {
@@ -826,10 +841,10 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
           }
         __syncwarp();
         for (int rho = blockIdx.x * 4 + (et >> 5); rho < rows && ok; rho += nct * 4)
-          quant_row_warp(ins[ib + rho / T], rho % T, H.eps, lane);
+          quant_row_warp(ins[ib + rho / T], rho % T, H.eps, lane, H.BN);
       } else {
         for (int rho = blockIdx.x; rho < rows && ok; rho += nct)
-          quant_row(ins[ib + rho / T], rho % T, H.eps, et, s_red_d, s_red_f, s_red_i);
+          quant_row(ins[ib + rho / T], rho % T, H.eps, et, H.BN, s_red_d, s_red_f, s_red_i);
       }
       fence_proxy_async_global();   // the codes are read by TMA (async proxy) in other CTAs
       named_bar_sync(1, kPEpi);
@@ -957,6 +972,28 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   }
 }
 
+// Re-tiles one projection's packed weights (canonical layout: [N x K/4] row-major) into
+// [tile][stage][128 rows x 128 B] blocks stored as the kernel's shared-memory image.  One CTA
+// per block; thread r copies row r of the block (a GLU tile takes 64 gated rows, then the 64
+// multiplier rows I apart).  Bytes past the end of a row are written as zeros.
+__global__ void __launch_bounds__(128) retile_weights_kernel(const uint8_t* __restrict__ Wp, int K,
+                                                             int N, int glu,
+                                                             uint8_t* __restrict__ Wt) {
+  const int row_bytes = K / 4;
+  const int nst = (row_bytes + kPWRow - 1) / kPWRow;
+  const int tile = static_cast<int>(blockIdx.x) / nst, st = static_cast<int>(blockIdx.x) % nst;
+  const int r = threadIdx.x;
+  const int row = glu ? (r < 64 ? tile * 64 + r : N / 2 + tile * 64 + (r - 64)) : tile * 128 + r;
+  const uint8_t* src = Wp + static_cast<int64_t>(row) * row_bytes + st * kPWRow;
+  uint8_t* dst = Wt + static_cast<int64_t>(blockIdx.x) * kPWStage + r * kPWRow;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (st * kPWRow + c * 16 < row_bytes) v = *reinterpret_cast<const uint4*>(src + c * 16);
+    *reinterpret_cast<uint4*>(dst + ((c ^ (r & 7)) << 4)) = v;
+  }
+}
+
 // ------------------------------------------------------------------------------ host planning
 struct Plan {
   std::vector<PIn> ins;
@@ -965,7 +1002,6 @@ struct Plan {
   std::vector<int32_t> ctaoff;
   PHeader h;
   size_t bytes = 0;
-  std::vector<CUtensorMap> maps;
   std::vector<std::pair<size_t, size_t>> in_buf;   // offset of A, and of gamma/rowsum, per input
   int BN = 0;
 };
@@ -1052,7 +1088,7 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
     q.ydt = p[i].ydt;
     q.in = proj_in[i];
     q.level = p[i].level;
-    q.wmap = i;
+    q.nst = static_cast<int32_t>((p[i].K / kPKB + kPSub - 1) / kPSub);
     P.projs.push_back(q);
     tile_base[i] = tiles;
     tiles += static_cast<int>(p[i].N / 128);
@@ -1127,25 +1163,31 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
   off = al(off + P.units.size() * sizeof(PUnit), 256);
   h.off_ctaoff = static_cast<int64_t>(off);
   off = al(off + P.ctaoff.size() * sizeof(int32_t), 256);
-  h.off_maps = static_cast<int64_t>(off);
-  off = al(off + (P.projs.size() + P.ins.size()) * sizeof(CUtensorMap), 256);
   h.off_tilectr = static_cast<int64_t>(off);
   off = al(off + static_cast<size_t>(tiles) * 4, 256);
   h.off_levelctr = static_cast<int64_t>(off);
   off = al(off + (2 * kMaxLevels + 2) * 4, 256);
+  // per input: its codes tiled for BN token rows (K x BN bytes), then gamma and the code sums
   for (size_t k = 0; k < P.ins.size(); ++k) {
     const size_t a_off = off;
-    off = al(off + static_cast<size_t>(T) * P.ins[k].K, 256);
+    off = al(off + static_cast<size_t>(P.BN) * P.ins[k].K, 256);
     const size_t v_off = off;
     off = al(off + static_cast<size_t>(T) * 8, 256);
     P.in_buf.push_back({a_off, v_off});
     P.ins[k].A = reinterpret_cast<int8_t*>(base + a_off);
     P.ins[k].gamma = reinterpret_cast<float*>(base + v_off);
     P.ins[k].rowsum = reinterpret_cast<int32_t*>(base + v_off + static_cast<size_t>(T) * 4);
-    P.ins[k].amap = n + static_cast<int32_t>(k);
+    P.ins[k].nst = static_cast<int32_t>((P.ins[k].K / kPKB + kPSub - 1) / kPSub);
   }
   h.off_part = static_cast<int64_t>(off);
   off = al(off + static_cast<size_t>(part_slots) * P.BN * 128 * 4, 256);
+  // the re-tiled packed weights of every projection: (N/128) tiles x nst stages x 16 KB
+  h.off_wt = static_cast<int64_t>(off);
+  for (size_t i = 0; i < P.projs.size(); ++i) {
+    PProj& q = P.projs[i];
+    q.Wt = reinterpret_cast<const uint8_t*>(base + off);
+    off = al(off + static_cast<size_t>(q.N / 128) * q.nst * kPWStage, 256);
+  }
   P.bytes = off;
   int k = 0;
   for (int L = 0; L <= n_levels; ++L) {
@@ -1213,23 +1255,6 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   st = build_plan(p, n, T, eps, reinterpret_cast<uintptr_t>(ws), nct, P);
   if (st != MMF_OK) return st;
   if (ws_bytes < P.bytes) return MMF_ERR_WORKSPACE;
-  // tensor maps: packed weights (box 64 rows x 128 B, 128-byte swizzle: one line of each row
-  // per stage; boxes reaching past the end of a row read zeros) and activation codes (box BN
-  // rows x 128 B, 128-byte swizzle)
-  P.maps.resize(P.projs.size() + P.ins.size());
-  for (size_t i = 0; i < P.projs.size(); ++i) {
-    const PProj& q = P.projs[i];
-    if (!make_tmap_2d_u8(&P.maps[i], q.Wp, static_cast<uint64_t>(q.K / 4), static_cast<uint64_t>(q.N),
-                         static_cast<uint64_t>(q.K / 4), kPWRow, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-      return MMF_ERR_CUDA;
-  }
-  for (size_t k = 0; k < P.ins.size(); ++k) {
-    const PIn& in = P.ins[k];
-    if (!make_tmap_2d_u8(&P.maps[P.projs.size() + k], in.A, static_cast<uint64_t>(in.K),
-                         static_cast<uint64_t>(T), static_cast<uint64_t>(in.K), kPKB,
-                         static_cast<uint32_t>(P.BN), CU_TENSOR_MAP_SWIZZLE_128B))
-      return MMF_ERR_CUDA;
-  }
   // host image of the plan region, copied in one stream-ordered copy; counters zeroed
   const size_t plan_end = static_cast<size_t>(P.h.off_levelctr) + (2 * kMaxLevels + 2) * 4;
   std::vector<uint8_t> img(plan_end, 0);
@@ -1238,15 +1263,21 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   std::memcpy(img.data() + P.h.off_proj, P.projs.data(), P.projs.size() * sizeof(PProj));
   std::memcpy(img.data() + P.h.off_units, P.units.data(), P.units.size() * sizeof(PUnit));
   std::memcpy(img.data() + P.h.off_ctaoff, P.ctaoff.data(), P.ctaoff.size() * sizeof(int32_t));
-  std::memcpy(img.data() + P.h.off_maps, P.maps.data(), P.maps.size() * sizeof(CUtensorMap));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // pageable source: the copy has consumed the host buffer when cudaMemcpyAsync returns
   if (cudaMemcpyAsync(ws, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return MMF_ERR_CUDA;
+  // the packed weights, re-tiled into the workspace once (they must not change afterwards)
+  for (size_t i = 0; i < P.projs.size(); ++i) {
+    const PProj& q = P.projs[i];
+    retile_weights_kernel<<<static_cast<unsigned>((q.N / 128) * q.nst), 128, 0, s>>>(
+        q.Wp, q.K, q.N, q.glu, const_cast<uint8_t*>(q.Wt));
+    if (cudaGetLastError() != cudaSuccess) return MMF_ERR_CUDA;
+  }
   // split tiles accumulate into zeroed int32 tiles (each run leaves them zeroed again)
-  if (P.bytes > static_cast<size_t>(P.h.off_part) &&
+  if (P.h.off_wt > P.h.off_part &&
       cudaMemsetAsync(static_cast<uint8_t*>(ws) + P.h.off_part, 0,
-                      P.bytes - static_cast<size_t>(P.h.off_part), s) != cudaSuccess)
+                      static_cast<size_t>(P.h.off_wt - P.h.off_part), s) != cudaSuccess)
     return MMF_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lk(g_runs_mu);

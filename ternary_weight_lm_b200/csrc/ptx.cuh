@@ -51,6 +51,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Tests two barrier phases in one statement, so that their latencies overlap (a satisfied
+// try_wait still costs a few hundred cycles before the next instruction can issue).
+__device__ __forceinline__ bool mbar_try_wait2(uint32_t bar1, uint32_t parity1, uint32_t bar2,
+                                               uint32_t parity2) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
+      "and.pred p, p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar1), "r"(parity1), "r"(bar2), "r"(parity2)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` of the barrier to complete.  Gives up after `limit_ns` of wall
 // time, or at once when *abort (shared) is set by another thread of the block; on a timeout
 // it sets *abort and ORs kStatusTimeout into *status.  Returns true when the phase completed.
@@ -92,6 +109,18 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t
                    reinterpret_cast<uint64_t>(m)),
                "r"(x), "r"(y)
                : "memory");
+}
+
+// Copies `bytes` contiguous bytes from global to shared memory (16-byte aligned addresses, size
+// a multiple of 16), completing on `bar` as a transaction count.  One large contiguous copy
+// streams at nearly the full HBM rate, unlike a tensor box of many short rows.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
 }
 
 // Brings `bytes` bytes at `p` into L2 (16-byte aligned address, size a multiple of 16).
