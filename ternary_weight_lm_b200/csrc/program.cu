@@ -541,7 +541,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   // group c % 3 (four slots, one per sub-block).  full(s): stage s's weight line and activation
   // sub-tiles landed.  empty(s): the unpack warps read its weights and the MMAs of that stage
   // completed -- one commit per stage, which also tells the unpack warps that the stage's slot
-  // group is free again (commits are costly on the MMA pipe, so there is no per-slot signal).
+  // group is free again (so there is no per-slot barrier to wait on).
   // afull(g): the unpack warps wrote slot group g.  accfull/accempty(b): accumulator b finished /
   // read by the epilogue.
   auto full = [&](int st) { return smem_u32(bars + st); };
