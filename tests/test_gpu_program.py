@@ -57,7 +57,7 @@ def _reference_outputs(projs):
     return dict(outs)
 
 
-@pytest.mark.parametrize("T", [1, 8, 17, 33, 64])
+@pytest.mark.parametrize("T", [1, 2, 3, 8, 17, 33, 64])
 def test_program_370m_block_matches_single_calls_and_oracle(T):
     projs, host = _block(1024, 2816, T, seed=T)
     prog = mmf.Program(projs, T)
