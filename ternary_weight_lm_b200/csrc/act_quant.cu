@@ -5,12 +5,13 @@
 // FusedBitLinear layers of the HGRNBit tree carry RMSNorm(eps=1e-08) inside the projection
 // ("matmulfreellm 評価 ...", section "HGRNBit という層構成を読む").
 //
-// One CTA of 128 threads per token row.  The row is read once from HBM with 16-byte loads and
-// kept in registers across the three block reductions it needs: sum of squares (double),
-// max |xhat| (float) and the sum of the int8 codes (int, used by the contraction to undo the
-// +1 offset of the packed weight codes).  Every rounding decision uses the same single-
-// precision operation sequence as the definition: ms = float(sum/K), r = sqrt(ms + eps),
-// inv = 1/r, xhat = (x * inv) * g, s = 127/gamma, q = round_half_even(xhat * s).
+// Many rows (prefill): one warp per row; few or very long rows: one 128-thread CTA per row.
+// The row is read once from HBM with 16-byte loads and kept in registers for the reductions it
+// needs: the sum of squares (double) together with max|x|, then (only with a norm weight)
+// max |xhat|, then the sum of the int8 codes (used by the contraction to undo the +1 offset of
+// the packed weight codes).  Every rounding decision uses the same single-precision operation
+// sequence as the definition: ms = float(sum/K), r = sqrt(ms + eps), inv = 1/r,
+// xhat = (x * inv) * g, s = 127/gamma, q = round_half_even(xhat * s).
 #include <cuda_fp16.h>
 
 #include "kernels.cuh"
@@ -47,19 +48,6 @@ struct Vec<__half> {
   }
 };
 
-__device__ __forceinline__ double block_sum_d(double v, double* sh) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 0) sh[w] = v;
-  __syncthreads();
-  double t = 0.0;
-#pragma unroll
-  for (int i = 0; i < kAqWarps; ++i) t += sh[i];
-  __syncthreads();
-  return t;
-}
-
 __device__ __forceinline__ float block_max_f(float v, float* sh) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -86,14 +74,57 @@ __device__ __forceinline__ int block_sum_i(int v, int* sh) {
   return t;
 }
 
-__device__ __forceinline__ uint32_t code_byte(float xh, float s) {
-  int q = __float2int_rn(__fmul_rn(xh, s));
-  q = max(-128, min(127, q));
-  return static_cast<uint32_t>(q) & 0xFFu;
+// q = round_half_even(y) saturated to [-128, 127], in one conversion; the low byte is the code.
+__device__ __forceinline__ int code_s8(float y) {
+  int q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(y));
+  return q;
 }
 
+// Four codes packed little-endian into one word (byte b = code b).
+__device__ __forceinline__ uint32_t pack4(int q0, int q1, int q2, int q3) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(q0), static_cast<uint32_t>(q1), 0x0040);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(q2), static_cast<uint32_t>(q3), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+// Codes of one 16-byte input vector: E/4 packed words; rs += the sum of the E signed codes.
+template <int E, bool kG>
+__device__ __forceinline__ void quantise_vec(const float (&v)[E], const float* gk, float inv_r,
+                                             float s, uint32_t (&w)[E / 4], int& rs) {
+#pragma unroll
+  for (int c = 0; c < E / 4; ++c) {
+    int q[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      // without a norm weight (x*inv)*1 is x*inv exactly
+      float xh = __fmul_rn(v[4 * c + b], inv_r);
+      if constexpr (kG) xh = __fmul_rn(xh, gk[4 * c + b]);
+      q[b] = code_s8(__fmul_rn(xh, s));
+    }
+    w[c] = pack4(q[0], q[1], q[2], q[3]);
+    rs = __dp4a(static_cast<int>(w[c]), 0x01010101, rs);
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void load_norm_weight(const float* g, int vi, float (&gk)[E]) {
+#pragma unroll
+  for (int e = 0; e < E; e += 4) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(g + vi * E + e));
+    gk[e] = t.x; gk[e + 1] = t.y; gk[e + 2] = t.z; gk[e + 3] = t.w;
+  }
+}
+
+// The row passes over the register-resident input:
+//   1. sum of squares (double) and, without a norm weight, max|x|;
+//   2. only with a norm weight (kG): gamma = max |(x*inv)*g| element by element;
+//   3. the codes and their sum.
+// Without a norm weight gamma = (max|x|)*inv exactly: round-to-nearest is monotone and odd, so
+// the largest |x*inv| is the rounded product of the largest |x| with inv.
+
 // MAXV = most 16-byte vectors one thread holds: K <= kAqThreads * MAXV * E.
-template <typename TIn, int MAXV, int MINB>
+template <typename TIn, int MAXV, int MINB, bool kG>
 __global__ void __launch_bounds__(kAqThreads, MINB)
 act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, float eps,
                  int8_t* __restrict__ A, float* __restrict__ gamma,
@@ -119,6 +150,7 @@ act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, 
     if (vi < nvec) raw[i] = __ldcs(xr + vi);   // streamed once: do not keep in L1
   }
   double ss = 0.0;
+  float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int vi = threadIdx.x + i * kAqThreads;
@@ -129,39 +161,48 @@ act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, 
       for (int e = 0; e < E; ++e) {
         const double d = static_cast<double>(v[e]);
         ss = __fma_rn(d, d, ss);   // d*d is exact in double: same as an add of the square
+        if constexpr (!kG) mx = fmaxf(mx, fabsf(v[e]));
       }
     }
   }
-  ss = block_sum_d(ss, sh_d);
+  // one barrier pair reduces both the sum of squares and max|x|
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if constexpr (!kG) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  {
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) { sh_d[w] = ss; sh_f[w] = mx; }
+    __syncthreads();
+    ss = 0.0;
+    mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kAqWarps; ++i) { ss += sh_d[i]; mx = fmaxf(mx, sh_f[i]); }
+    __syncthreads();
+  }
   const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
   const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 
-  auto norm_weight = [&](int vi, float (&gk)[E]) {
-    if (g != nullptr) {
+  float amax;
+  if constexpr (kG) {
+    amax = 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; e += 4) {
-        const float4 t = __ldg(reinterpret_cast<const float4*>(g + vi * E + e));
-        gk[e] = t.x; gk[e + 1] = t.y; gk[e + 2] = t.z; gk[e + 3] = t.w;
+    for (int i = 0; i < MAXV; ++i) {
+      const int vi = threadIdx.x + i * kAqThreads;
+      if (vi < nvec) {
+        float v[E], gk[E];
+        V::widen(raw[i], v);
+        load_norm_weight(g, vi, gk);
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), gk[e])));
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) gk[e] = 1.0f;
     }
-  };
-
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
-    const int vi = threadIdx.x + i * kAqThreads;
-    if (vi < nvec) {
-      float v[E], gk[E];
-      V::widen(raw[i], v);
-      norm_weight(vi, gk);
-#pragma unroll
-      for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), gk[e])));
-    }
+    amax = block_max_f(amax, sh_f);
+  } else {
+    amax = __fmul_rn(mx, inv_r);
   }
-  amax = block_max_f(amax, sh_f);
   const float gm = fmaxf(amax, 1e-5f);
   const float s = __fdiv_rn(127.0f, gm);
 
@@ -173,20 +214,9 @@ act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, 
     if (vi < nvec) {
       float v[E], gk[E];
       V::widen(raw[i], v);
-      norm_weight(vi, gk);
+      if constexpr (kG) load_norm_weight(g, vi, gk);
       uint32_t w[E / 4];
-#pragma unroll
-      for (int c = 0; c < E / 4; ++c) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float xh = __fmul_rn(__fmul_rn(v[4 * c + b], inv_r), gk[4 * c + b]);
-          const uint32_t cb = code_byte(xh, s);
-          rs += static_cast<int>(static_cast<int8_t>(cb));
-          word |= cb << (8 * b);
-        }
-        w[c] = word;
-      }
+      quantise_vec<E, kG>(v, gk, inv_r, s, w, rs);
       if constexpr (E == 8) {
         *reinterpret_cast<uint2*>(ar + vi * E) = make_uint2(w[0], w[1]);
       } else {
@@ -205,7 +235,7 @@ act_quant_kernel(const TIn* __restrict__ x, int K, const float* __restrict__ g, 
 // every reduction a warp shuffle, no block barriers.  Same arithmetic, same op order.
 constexpr int kWarpRowsPerCta = 8;
 
-template <typename TIn, int VPL>
+template <typename TIn, int VPL, bool kG>
 __global__ void __launch_bounds__(32 * kWarpRowsPerCta)
 act_quant_warp_kernel(const TIn* __restrict__ x, int64_t T, int K, const float* __restrict__ g,
                       float eps, int8_t* __restrict__ A, float* __restrict__ gamma,
@@ -227,6 +257,7 @@ act_quant_warp_kernel(const TIn* __restrict__ x, int64_t T, int K, const float* 
     if (vi < nvec) raw[i] = __ldcs(xr + vi);
   }
   double ss = 0.0;
+  float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     if (lane + 32 * i < nvec) {
@@ -236,40 +267,38 @@ act_quant_warp_kernel(const TIn* __restrict__ x, int64_t T, int K, const float* 
       for (int e = 0; e < E; ++e) {
         const double d = static_cast<double>(v[e]);
         ss = __fma_rn(d, d, ss);
+        if constexpr (!kG) mx = fmaxf(mx, fabsf(v[e]));
       }
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if constexpr (!kG) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
   const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
   const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 
-  auto norm_weight = [&](int vi, float (&gk)[E]) {
-    if (g != nullptr) {
+  float amax;
+  if constexpr (kG) {
+    amax = 0.0f;
 #pragma unroll
-      for (int e = 0; e < E; e += 4) {
-        const float4 t = __ldg(reinterpret_cast<const float4*>(g + vi * E + e));
-        gk[e] = t.x; gk[e + 1] = t.y; gk[e + 2] = t.z; gk[e + 3] = t.w;
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = lane + 32 * i;
+      if (vi < nvec) {
+        float v[E], gk[E];
+        V::widen(raw[i], v);
+        load_norm_weight(g, vi, gk);
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+          amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), gk[e])));
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) gk[e] = 1.0f;
     }
-  };
-  float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int vi = lane + 32 * i;
-    if (vi < nvec) {
-      float v[E], gk[E];
-      V::widen(raw[i], v);
-      norm_weight(vi, gk);
-#pragma unroll
-      for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), gk[e])));
-    }
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  } else {
+    amax = __fmul_rn(mx, inv_r);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float gm = fmaxf(amax, 1e-5f);
   const float s = __fdiv_rn(127.0f, gm);
 
@@ -281,20 +310,9 @@ act_quant_warp_kernel(const TIn* __restrict__ x, int64_t T, int K, const float* 
     if (vi < nvec) {
       float v[E], gk[E];
       V::widen(raw[i], v);
-      norm_weight(vi, gk);
+      if constexpr (kG) load_norm_weight(g, vi, gk);
       uint32_t w[E / 4];
-#pragma unroll
-      for (int c = 0; c < E / 4; ++c) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const float xh = __fmul_rn(__fmul_rn(v[4 * c + b], inv_r), gk[4 * c + b]);
-          const uint32_t cb = code_byte(xh, s);
-          rs += static_cast<int>(static_cast<int8_t>(cb));
-          word |= cb << (8 * b);
-        }
-        w[c] = word;
-      }
+      quantise_vec<E, kG>(v, gk, inv_r, s, w, rs);
       if constexpr (E == 8) {
         *reinterpret_cast<uint2*>(ar + vi * E) = make_uint2(w[0], w[1]);
       } else {
@@ -329,6 +347,52 @@ rowsum_kernel(const int8_t* __restrict__ A, int K, int32_t* __restrict__ rowsum)
   if (threadIdx.x == 0) rowsum[row] = s;
 }
 
+template <bool kG>
+cudaError_t launch_act_quant_t(const cudaLaunchConfig_t& base, const void* x, int xdt, int64_t T,
+                               int K, const float* g, float eps, int8_t* A, float* gamma,
+                               int32_t* rowsum) {
+  cudaLaunchConfig_t cfg = base;
+  const int e = xdt == kInF16 ? 8 : 4;          // elements per 16-byte vector
+  const int nvec = K / e;
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  const float* xf = reinterpret_cast<const float*>(x);
+  if (nvec <= 32 * 24 && T >= 256) {
+    // many rows (prefill): one warp per row; few rows (decode) keep a CTA per row so each
+    // row's loads and reductions spread over more threads
+    cfg.gridDim = dim3(static_cast<unsigned>((T + kWarpRowsPerCta - 1) / kWarpRowsPerCta));
+    cfg.blockDim = dim3(32 * kWarpRowsPerCta);
+    if (xdt == kInF16) {
+      if (nvec <= 32 * 8)
+        return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<__half, 8, kG>, xh, T, K, g, eps,
+                                  A, gamma, rowsum);
+      if (nvec <= 32 * 16)
+        return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<__half, 16, kG>, xh, T, K, g, eps,
+                                  A, gamma, rowsum);
+      return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<__half, 24, kG>, xh, T, K, g, eps,
+                                A, gamma, rowsum);
+    }
+    if (nvec <= 32 * 8)
+      return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<float, 8, kG>, xf, T, K, g, eps, A,
+                                gamma, rowsum);
+    if (nvec <= 32 * 16)
+      return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<float, 16, kG>, xf, T, K, g, eps, A,
+                                gamma, rowsum);
+    return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<float, 24, kG>, xf, T, K, g, eps, A,
+                              gamma, rowsum);
+  }
+  // few or long rows: one 128-thread CTA per row
+  cfg.gridDim = dim3(static_cast<unsigned>(T));
+  cfg.blockDim = dim3(kAqThreads);
+  if (xdt == kInF16) {
+    // 8 halves per vector: K <= 128 * 8 * 8 = 8192
+    return cudaLaunchKernelEx(&cfg, act_quant_kernel<__half, 8, 8, kG>, xh, K, g, eps, A, gamma,
+                              rowsum);
+  }
+  // 4 floats per vector: K <= 128 * 16 * 4 = 8192
+  return cudaLaunchKernelEx(&cfg, act_quant_kernel<float, 16, 4, kG>, xf, K, g, eps, A, gamma,
+                            rowsum);
+}
+
 }  // namespace
 
 cudaError_t launch_act_quant(const void* x, int xdt, int64_t T, int K, const float* g, float eps,
@@ -340,37 +404,8 @@ cudaError_t launch_act_quant(const void* x, int xdt, int64_t T, int K, const flo
   cfg.stream = s;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  const int e = xdt == kInF16 ? 8 : 4;          // elements per 16-byte vector
-  const int nvec = K / e;
-  if (nvec <= 32 * 16 && T >= 256) {
-    // many short rows (prefill): one warp per row; few rows (decode) keep a CTA per row so
-    // each row's loads and reductions spread over more threads
-    cfg.gridDim = dim3(static_cast<unsigned>((T + kWarpRowsPerCta - 1) / kWarpRowsPerCta));
-    cfg.blockDim = dim3(32 * kWarpRowsPerCta);
-    if (xdt == kInF16) {
-      if (nvec <= 32 * 8)
-        return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<__half, 8>,
-                                  reinterpret_cast<const __half*>(x), T, K, g, eps, A, gamma, rowsum);
-      return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<__half, 16>,
-                                reinterpret_cast<const __half*>(x), T, K, g, eps, A, gamma, rowsum);
-    }
-    if (nvec <= 32 * 8)
-      return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<float, 8>,
-                                reinterpret_cast<const float*>(x), T, K, g, eps, A, gamma, rowsum);
-    return cudaLaunchKernelEx(&cfg, act_quant_warp_kernel<float, 16>,
-                              reinterpret_cast<const float*>(x), T, K, g, eps, A, gamma, rowsum);
-  }
-  // long rows: one 128-thread CTA per row
-  cfg.gridDim = dim3(static_cast<unsigned>(T));
-  cfg.blockDim = dim3(kAqThreads);
-  if (xdt == kInF16) {
-    // 8 halves per vector: K <= 128 * 8 * 8 = 8192
-    return cudaLaunchKernelEx(&cfg, act_quant_kernel<__half, 8, 8>,
-                              reinterpret_cast<const __half*>(x), K, g, eps, A, gamma, rowsum);
-  }
-  // 4 floats per vector: K <= 128 * 16 * 4 = 8192
-  return cudaLaunchKernelEx(&cfg, act_quant_kernel<float, 16, 4>,
-                            reinterpret_cast<const float*>(x), K, g, eps, A, gamma, rowsum);
+  if (g != nullptr) return launch_act_quant_t<true>(cfg, x, xdt, T, K, g, eps, A, gamma, rowsum);
+  return launch_act_quant_t<false>(cfg, x, xdt, T, K, g, eps, A, gamma, rowsum);
 }
 
 cudaError_t launch_rowsum(const int8_t* A, int64_t T, int K, int32_t* rowsum, cudaStream_t s) {

@@ -70,6 +70,11 @@ def test_ternary_encode_given_beta():
     (64, 2816, np.float16, 0.0, False), (300, 2048, np.float16, 0.01, False),
     (16, 256, np.float32, 0.0, False), (9, 7040, np.float16, 0.01, True),
     (5, 8192, np.float32, 0.0, True), (3, 8192, np.float16, 0.0, False),
+    # T >= 256: one warp per row, 8 / 16 / 24 vectors per lane, with and without a norm weight
+    (300, 2048, np.float16, 0.01, True), (264, 4096, np.float16, 0.0, False),
+    (260, 5632, np.float16, 0.01, True), (257, 5632, np.float16, 0.0, False),
+    (300, 1024, np.float32, 0.01, True), (256, 2816, np.float32, 0.0, False),
+    (259, 2816, np.float32, 0.0, True),
 ])
 def test_quantize_activations(T, K, dt, outliers, gw):
     x = synth.activations(T * 7 + K, f"aq{T}x{K}", T, K, dtype=dt, outlier_frac=outliers)
