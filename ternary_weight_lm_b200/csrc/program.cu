@@ -100,6 +100,7 @@ struct PHeader {
   int32_t pad[3];
   int64_t off_in, off_proj, off_units, off_ctaoff, off_wt, off_tilectr, off_levelctr, off_part;
   int32_t in_begin[kMaxLevels + 1];
+  int32_t qgroup[kMaxLevels];   // epilogue threads per input row in level L's quantisation
 };
 
 template <int BN>
@@ -181,84 +182,128 @@ __device__ __forceinline__ void widen16(const uint4& a, int xdt, float (&v)[8], 
   }
 }
 
-// The 128 epilogue threads quantise row t of input `in` together: the same operations, in the
-// same order, as the activation pre-pass kernel (mean of squares in double, rounded once;
-// inv = 1/sqrt(ms+eps); xhat = (x*inv)*g; gamma = max|xhat| floored at 1e-5;
-// q = rne(xhat * (127/gamma))).  The row is read once (ld.global.cg: this launch may have
-// written it) into registers, at most 8 vectors of 16 bytes per thread (K <= 8192 fp16 /
-// 4096 fp32).  red_d/red_f/red_i: per-warp partials in shared memory.
-__device__ void quant_row(const PIn in, int t, float eps, int et, int bn, double* red_d,
-                          float* red_f, int* red_i) {
+// A group of G epilogue threads (G = 32, 64 or 128: one, two or all four warps) quantises row
+// t of input `in` with the same operations per element as the activation pre-pass kernel
+// (mean of squares in double, rounded once; inv = 1/sqrt(ms+eps); xhat = (x*inv)*g;
+// gamma = max|xhat| floored at 1e-5; q = rne(xhat * (127/gamma)), saturated to int8).  The
+// row is read once (ld.global.cg: this launch may have written it) into registers, at most 8
+// vectors of 16 bytes per thread, so nvec <= 8*G; thread gt holds vectors gt, gt+G, ...
+// Without a norm weight gamma = (max|x|)*inv exactly: round-to-nearest is monotone and odd, so
+// the largest |x*inv| is the rounded product of the largest |x| with inv.
+// Partials cross warps through red_d/red_f/red_i (indexed by the epilogue warp 0-3) under
+// named barrier `bar` of G threads; only the order in which the per-thread sums of squares
+// are added depends on G, which can move the double sum by an ulp, far below the float
+// rounding of the mean.
+__device__ __forceinline__ int code_s8(float y) {
+  int q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(y));
+  return q;
+}
+
+__device__ __forceinline__ uint32_t pack4(int q0, int q1, int q2, int q3) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(q0), static_cast<uint32_t>(q1), 0x0040);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(q2), static_cast<uint32_t>(q3), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+__device__ void quant_row_g(const PIn in, int t, float eps, int gt, int G, int bar, int w,
+                            int bn, double* red_d, float* red_f, int* red_i) {
   constexpr int kVmax = 8;
   const int K = in.K;
   const int E = in.xdt == kInF16 ? 8 : 4;
   const int nvec = K / E;
-  const int lane = et & 31, w = et >> 5;
+  const int lane = gt & 31;
+  const int w0 = w - (gt >> 5);                 // first epilogue warp of the group
+  const int nw = G >> 5;
   const uint4* xr = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(in.x) +
                                                    static_cast<int64_t>(t) * K * (E == 8 ? 2 : 4));
   uint4 raw[kVmax];
 #pragma unroll
   for (int i = 0; i < kVmax; ++i) {
-    const int vi = et + kPEpi * i;
+    const int vi = gt + G * i;
     if (vi < nvec) raw[i] = __ldcg(xr + vi);
   }
+  const bool has_g = in.g != nullptr;
   double ss = 0.0;
+  float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < kVmax; ++i) {
-    if (et + kPEpi * i < nvec) {
+    if (gt + G * i < nvec) {
       float v[8];
       int n;
       widen16(raw[i], in.xdt, v, n);
       for (int e = 0; e < n; ++e) {
         const double d = static_cast<double>(v[e]);
         ss = __fma_rn(d, d, ss);
+        mx = fmaxf(mx, fabsf(v[e]));
       }
     }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) red_d[w] = ss;
-  named_bar_sync(1, kPEpi);
-  ss = red_d[0] + red_d[1] + red_d[2] + red_d[3];
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (nw > 1) {
+    if (lane == 0) {
+      red_d[w] = ss;
+      red_f[w] = mx;
+    }
+    named_bar_sync(bar, G);
+    ss = red_d[w0];
+    mx = red_f[w0];
+    for (int j = 1; j < nw; ++j) {
+      ss += red_d[w0 + j];
+      mx = fmaxf(mx, red_f[w0 + j]);
+    }
+  }
   const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
   const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
   float amax = 0.0f;
+  if (!has_g) {
+    amax = __fmul_rn(mx, inv_r);
+  } else {
 #pragma unroll
-  for (int i = 0; i < kVmax; ++i) {
-    const int vi = et + kPEpi * i;
-    if (vi < nvec) {
-      float v[8];
-      int n;
-      widen16(raw[i], in.xdt, v, n);
-      for (int e = 0; e < n; ++e) {
-        const float gk = in.g ? __ldg(in.g + vi * E + e) : 1.0f;
-        amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), gk)));
+    for (int i = 0; i < kVmax; ++i) {
+      const int vi = gt + G * i;
+      if (vi < nvec) {
+        float v[8];
+        int n;
+        widen16(raw[i], in.xdt, v, n);
+        for (int e = 0; e < n; ++e)
+          amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), __ldg(in.g + vi * E + e))));
       }
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (lane == 0) red_f[w] = amax;
-  named_bar_sync(1, kPEpi);
-  amax = fmaxf(fmaxf(red_f[0], red_f[1]), fmaxf(red_f[2], red_f[3]));
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (nw > 1) {
+      if (lane == 0) red_f[4 + w] = amax;
+      named_bar_sync(bar, G);
+      amax = red_f[4 + w0];
+      for (int j = 1; j < nw; ++j) amax = fmaxf(amax, red_f[4 + w0 + j]);
+    }
+  }
   const float gm = fmaxf(amax, 1e-5f);
   const float s = __fdiv_rn(127.0f, gm);
   int rs = 0;
 #pragma unroll
   for (int i = 0; i < kVmax; ++i) {
-    const int vi = et + kPEpi * i;
+    const int vi = gt + G * i;
     if (vi < nvec) {
       float v[8];
       int n;
       widen16(raw[i], in.xdt, v, n);
-      uint32_t wd[2] = {0u, 0u};
-      for (int e = 0; e < n; ++e) {
-        const float gk = in.g ? __ldg(in.g + vi * E + e) : 1.0f;
-        const float xh = __fmul_rn(__fmul_rn(v[e], inv_r), gk);
-        int q = __float2int_rn(__fmul_rn(xh, s));
-        q = max(-128, min(127, q));
-        rs += q;
-        wd[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (e & 3));
+      uint32_t wd[2];
+      for (int c = 0; c < n / 4; ++c) {
+        int q[4];
+        for (int b = 0; b < 4; ++b) {
+          const int e = 4 * c + b;
+          float xh = __fmul_rn(v[e], inv_r);    // (x*inv)*1 is x*inv exactly
+          if (has_g) xh = __fmul_rn(xh, __ldg(in.g + vi * E + e));
+          q[b] = code_s8(__fmul_rn(xh, s));
+        }
+        wd[c] = pack4(q[0], q[1], q[2], q[3]);
+        rs = __dp4a(static_cast<int>(wd[c]), 0x01010101, rs);
       }
       if (E == 8)
         *reinterpret_cast<uint2*>(in.A + a_tiled(t, vi * 8, bn)) = make_uint2(wd[0], wd[1]);
@@ -268,128 +313,18 @@ __device__ void quant_row(const PIn in, int t, float eps, int et, int bn, double
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
-  if (lane == 0) red_i[w] = rs;
-  named_bar_sync(1, kPEpi);
-  if (et == 0) {
-    in.gamma[t] = gm;
-    in.rowsum[t] = red_i[0] + red_i[1] + red_i[2] + red_i[3];
+  if (nw > 1) {
+    if (lane == 0) red_i[w] = rs;
+    named_bar_sync(bar, G);
+    if (gt == 0)
+      for (int j = 1; j < nw; ++j) rs += red_i[w0 + j];
   }
-  named_bar_sync(1, kPEpi);   // the scratch is reused by the next row
-}
-
-// One warp quantises row t of input `in` alone, with the same operations per element as
-// quant_row (only the order in which the per-lane sums of squares are added differs, which can
-// move the double sum by an ulp, far below the float rounding of the mean).  Used when a level
-// has more rows than CTAs, so that each CTA's four epilogue warps work on four rows at once.
-// The row is streamed kQW vectors of 16 bytes per lane at a time (any K; few registers, as
-// the kernel's ten warps leave 168 per thread), in passes over L2:
-//   1. sum of squares (double) and, without a norm weight, max|x|;
-//   2. only with a norm weight: gamma = max |(x*inv)*g| element by element;
-//   3. the codes.
-// Without a norm weight gamma = (max|x|)*inv exactly: rounding is monotone, so the largest
-// |x*inv| comes from the largest |x| (and *1.0f is exact).
-constexpr int kQW = 2;
-__device__ void quant_row_warp(const PIn in, int t, float eps, int lane, int bn) {
-  const int K = in.K;
-  const int E = in.xdt == kInF16 ? 8 : 4;
-  const int nvec = K / E;
-  const uint4* xr = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(in.x) +
-                                                   static_cast<int64_t>(t) * K * (E == 8 ? 2 : 4));
-  double ss = 0.0;
-  float mx = 0.0f;
-#pragma unroll 1
-  for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
-    uint4 raw[kQW];
-#pragma unroll
-    for (int i = 0; i < kQW; ++i) {
-      const int vi = v0 + lane + 32 * i;
-      if (vi < nvec) raw[i] = __ldcg(xr + vi);
-    }
-#pragma unroll
-    for (int i = 0; i < kQW; ++i) {
-      if (v0 + lane + 32 * i < nvec) {
-        float v[8];
-        int n;
-        widen16(raw[i], in.xdt, v, n);
-        for (int e = 0; e < n; ++e) {
-          const double d = static_cast<double>(v[e]);
-          ss = __fma_rn(d, d, ss);
-          mx = fmaxf(mx, fabsf(v[e]));
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float ms = __double2float_rn(__ddiv_rn(ss, static_cast<double>(K)));
-  const float inv_r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
-  float amax = 0.0f;
-  if (in.g == nullptr) {
-    amax = __fmul_rn(mx, inv_r);
-  } else {
-  #pragma unroll 1
-  for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
-      uint4 raw[kQW];
-#pragma unroll
-      for (int i = 0; i < kQW; ++i) {
-        const int vi = v0 + lane + 32 * i;
-        if (vi < nvec) raw[i] = __ldcg(xr + vi);
-      }
-#pragma unroll
-      for (int i = 0; i < kQW; ++i) {
-        const int vi = v0 + lane + 32 * i;
-        if (vi < nvec) {
-          float v[8];
-          int n;
-          widen16(raw[i], in.xdt, v, n);
-          for (int e = 0; e < n; ++e)
-            amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(v[e], inv_r), __ldg(in.g + vi * E + e))));
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float gm = fmaxf(amax, 1e-5f);
-  const float s = __fdiv_rn(127.0f, gm);
-  int rs = 0;
-#pragma unroll 1
-  for (int v0 = 0; v0 < nvec; v0 += 32 * kQW) {
-    uint4 raw[kQW];
-#pragma unroll
-    for (int i = 0; i < kQW; ++i) {
-      const int vi = v0 + lane + 32 * i;
-      if (vi < nvec) raw[i] = __ldcg(xr + vi);
-    }
-#pragma unroll
-    for (int i = 0; i < kQW; ++i) {
-      const int vi = v0 + lane + 32 * i;
-      if (vi < nvec) {
-        float v[8];
-        int n;
-        widen16(raw[i], in.xdt, v, n);
-        uint32_t wd[2] = {0u, 0u};
-        for (int e = 0; e < n; ++e) {
-          const float gk = in.g ? __ldg(in.g + vi * E + e) : 1.0f;
-          const float xh = __fmul_rn(__fmul_rn(v[e], inv_r), gk);
-          int q = __float2int_rn(__fmul_rn(xh, s));
-          q = max(-128, min(127, q));
-          rs += q;
-          wd[e >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (e & 3));
-        }
-        if (E == 8)
-          *reinterpret_cast<uint2*>(in.A + a_tiled(t, vi * 8, bn)) = make_uint2(wd[0], wd[1]);
-        else
-          *reinterpret_cast<uint32_t*>(in.A + a_tiled(t, vi * 4, bn)) = wd[0];
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
-  if (lane == 0) {
+  if (gt == 0) {
     in.gamma[t] = gm;
     in.rowsum[t] = rs;
   }
+  // red_* are written again only after the next row's first barrier, which every thread of
+  // the group reaches after its reads above
 }
 
 __device__ __forceinline__ void unpack_word4(uint32_t w, uint32_t* out) {
@@ -534,7 +469,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   __shared__ int s_flag;
   __shared__ int s_qflag;
   __shared__ double s_red_d[4];
-  __shared__ float s_red_f[4];
+  __shared__ float s_red_f[8];
   __shared__ int s_red_i[4];
 
   // Stage counter c (per CTA, over all its units) uses shared-memory stage c % S and TMEM slot
@@ -830,22 +765,22 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       // 1. quantise a share of this level's input rows (the 128 threads take one row at a time)
       const int ib = H.in_begin[L], ie = H.in_begin[L + 1];
       const int rows = (ie - ib) * T;
-      if (rows > nct) {   // more rows than CTAs: one row per warp, four at once
-        // first every row this warp will quantise is requested into L2 at once
-        if (lane == 0)
-          for (int rho = blockIdx.x * 4 + (et >> 5); rho < rows; rho += nct * 4) {
-            const PIn& in = ins[ib + rho / T];
-            const int rb = in.K * (in.xdt == kInF16 ? 2 : 4);
-            bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(in.x) + static_cast<int64_t>(rho % T) * rb,
-                             static_cast<uint32_t>(rb));
-          }
-        __syncwarp();
-        for (int rho = blockIdx.x * 4 + (et >> 5); rho < rows && ok; rho += nct * 4)
-          quant_row_warp(ins[ib + rho / T], rho % T, H.eps, lane, H.BN);
-      } else {
-        for (int rho = blockIdx.x; rho < rows && ok; rho += nct)
-          quant_row(ins[ib + rho / T], rho % T, H.eps, et, H.BN, s_red_d, s_red_f, s_red_i);
-      }
+      // a group of G threads per row, G fixed per level at plan time: the largest group that
+      // still finishes the level's rows in the fewest rounds, each row read in one pass
+      const int G = H.qgroup[L];
+      const int R = kPEpi / G;                    // rows in flight per CTA
+      const int gid = et / G, gt = et % G;
+      // first every row this group will quantise is requested into L2 at once
+      if (gt == 0)
+        for (int rho = blockIdx.x * R + gid; rho < rows; rho += nct * R) {
+          const PIn& in = ins[ib + rho / T];
+          const int rb = in.K * (in.xdt == kInF16 ? 2 : 4);
+          bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(in.x) + static_cast<int64_t>(rho % T) * rb,
+                           static_cast<uint32_t>(rb));
+        }
+      for (int rho = blockIdx.x * R + gid; rho < rows && ok; rho += nct * R)
+        quant_row_g(ins[ib + rho / T], rho % T, H.eps, gt, G, G == kPEpi ? 1 : 2 + gid, et >> 5,
+                    H.BN, s_red_d, s_red_f, s_red_i);
       fence_proxy_async_global();   // the codes are read by TMA (async proxy) in other CTAs
       named_bar_sync(1, kPEpi);
       if (et == 0) {
@@ -1195,6 +1130,26 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
     h.in_begin[L] = k;
   }
   h.in_begin[n_levels] = static_cast<int32_t>(P.ins.size());
+  // quantisation group per level: at most 8 vectors of 16 bytes per thread, then the fewest
+  // rounds of rows over the CTAs, then the most threads per row (shortest row latency)
+  for (int L = 0; L < n_levels; ++L) {
+    int nvec = 0;
+    for (int i = h.in_begin[L]; i < h.in_begin[L + 1]; ++i)
+      nvec = std::max(nvec, P.ins[i].K / (P.ins[i].xdt == kInF16 ? 8 : 4));
+    const int64_t rows = static_cast<int64_t>(h.in_begin[L + 1] - h.in_begin[L]) * T;
+    int best = kPEpi;
+    int64_t best_rounds = -1;
+    for (int G = kPEpi; G >= 32; G >>= 1) {
+      if (nvec > 8 * G) break;
+      const int64_t slots = static_cast<int64_t>(nct) * (kPEpi / G);
+      const int64_t rounds = (rows + slots - 1) / slots;
+      if (best_rounds < 0 || rounds < best_rounds) {
+        best = G;
+        best_rounds = rounds;
+      }
+    }
+    h.qgroup[L] = best;
+  }
   return MMF_OK;
 }
 
