@@ -42,8 +42,9 @@
 namespace mmf {
 namespace {
 
-// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 unpack, 6-9 quantise + epilogue.
-constexpr int kPThreads = 320;
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 and 10-13 unpack (even and odd stages),
+// 6-9 quantise + epilogue.
+constexpr int kPThreads = 448;
 constexpr int kPEpi = 128;
 constexpr int kPEpiT0 = 192;               // first epilogue thread
 constexpr int kPKB = 128;                  // K per TMEM slot (one sub-block)
@@ -560,7 +561,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       Cur wc, ac;
       load_cur(wc, u_begin);
       ac = wc;
-      int64_t wi = 0, ai = 0;
+      uint32_t wi = 0, ai = 0;             // 32-bit: cheap % and /
       int q_level = -1;
       bool ok = true;
       auto issue_act = [&]() {
@@ -610,7 +611,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       // them now (the workspace buffer is valid memory), so that every started stage
       // completes; then wait until every copy this thread started has landed.
       while (ai < wi && ac.ui < u_end) issue_act();
-      for (int64_t i = wi > S ? wi - S : 0; i < wi; ++i)
+      for (uint32_t i = wi > S ? wi - S : 0; i < wi; ++i)
         mbar_wait_bounded(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1),
                           kPDrainNs, nullptr, status);
     }
@@ -620,7 +621,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
     // lane issues each MMA and commit.
     constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
     const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
-    int64_t c = 0;                       // stage counter
+    uint32_t c = 0;                      // stage counter (32-bit: cheap % and /)
     bool ok = true;
     int n = 0;
     int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
@@ -681,25 +682,29 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
     tc_commit_warp(drainbar);
     mbar_wait_bounded(drainbar, 0u, kPDrainNs, nullptr, status);
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 6 || warp >= 10) {
     // ------------------------------------------------------------------ unpack
     // Each lane owns one tile row (= TMEM lane): per stage it reads its row's 128-byte weight
-    // line once and unpacks its sub-blocks (32 bytes, 128 codes each) into TMEM slots.
+    // line once and unpacks its sub-blocks (32 bytes, 128 codes each) into TMEM slots.  Two
+    // sets of four warps take alternate stages, so that one set's store and barrier latencies
+    // overlap the other's unpacking.
+    const int set = warp >= 10 ? 1 : 0;
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-    int64_t c = 0;                       // stage counter
+    uint32_t c = 0;                      // stage counter (32-bit: cheap % and /)
     bool ok = true;
     for (int ui = u_begin; ui < u_end && ok; ++ui) {
       const int nkb = units[ui].nkb;
       for (int k = 0; k < nkb; k += kPSub, ++c) {
+        if (static_cast<int>(c & 1) != set) continue;
         const int nsub = min(kPSub, nkb - k);
         const int st = static_cast<int>(c % S);
         const int gi = static_cast<int>(c % kPGroups);
         // Both conditions of this stage (its data landed; its slot group is free, see below)
         // are tested in one statement first; the bounded waits run only if one is not met.
-        const int64_t cp = c - kPGroups;
-        const bool both = cp >= 0 && mbar_try_wait2(full(st), static_cast<uint32_t>((c / S) & 1),
+        const uint32_t cp = c - kPGroups;   // valid when c >= kPGroups
+        const bool both = c >= kPGroups && mbar_try_wait2(full(st), static_cast<uint32_t>((c / S) & 1),
                                                      empty(static_cast<int>(cp % S)),
                                                      static_cast<uint32_t>((cp / S) & 1));
         bool w = both || mbar_wait_bounded(full(st), static_cast<uint32_t>((c / S) & 1),
@@ -718,8 +723,8 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         if (lane == 0) mbar_arrive(empty(st));
         // slot group gi was last read by the MMAs of stage c - 3: their commit completed
         // empty((c - 3) % S).  (That barrier cannot have moved a further phase on: it needs
-        // this warp's arrival for stage c - 3 + S first.)
-        if (cp >= 0 && !both) {
+        // the arrivals for stage c - 3 + S, which come after this stage's.)
+        if (c >= kPGroups && !both) {
           w = mbar_wait_bounded(empty(static_cast<int>(cp % S)), static_cast<uint32_t>((cp / S) & 1),
                                 limit_ns, abort_flag, status);
           if (!__all_sync(0xFFFFFFFFu, w)) {
