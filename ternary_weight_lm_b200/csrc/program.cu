@@ -95,11 +95,26 @@ struct PUnit {
   int32_t proj, tile, kb0, nkb, split, nsplit, tile_id, part_off;
 };
 
+// What the epilogue needs of a unit, flattened at plan time and staged in shared memory by
+// the epilogue threads (kERecMax units at a time, one load each), so that starting a unit
+// costs no chain of dependent L2 round trips (unit -> projection -> input -> scales).
+struct PERec {
+  void* y;
+  const float* beta;
+  const float* gamma;
+  const int32_t* rowsum;
+  int32_t tile, nsplit, part_off, tile_id;
+  int32_t nkb, N, level, flags;   // flags: glu | ydt << 1
+};
+static_assert(sizeof(PERec) == 64, "four 16-byte words");
+constexpr int kERecMax = 128;
+
 struct PHeader {
   int32_t n_proj, n_in, n_levels, n_ctas, n_units, T, BN, n_tiles;
   float eps;
   int32_t pad[3];
   int64_t off_in, off_proj, off_units, off_ctaoff, off_wt, off_tilectr, off_levelctr, off_part;
+  int64_t off_erec;
   int32_t in_begin[kMaxLevels + 1];
   int32_t qgroup[kMaxLevels];   // epilogue threads per input row in level L's quantisation
 };
@@ -113,11 +128,12 @@ struct PCfg {
   static constexpr int kXbuf = kCh * 64 * 4;      // GLU exchange: multiplier half, fp32
   static constexpr int kTok = 8 * 64;             // per-token scale and code sum
   static constexpr int kOst = BN * 128 * 2;       // fp16 output staging [token][column]
-  static constexpr int kFixed = 1024 + 1024 + kXbuf + kTok + kOst + 64;
+  static constexpr int kERec = kERecMax * 64;     // staged epilogue records
+  static constexpr int kFixed = 1024 + 1024 + kXbuf + kTok + kOst + kERec + 64;
   static constexpr int kStagesFit = (227 * 1024 - 512 - kFixed) / kStage;
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
   static constexpr int kBar = (8 * (2 * kStages + kPGroups + 5) + 127) / 128 * 128;
-  static constexpr int kSmem = 1024 + kStages * kStage + kBar + kXbuf + kTok + kOst + 64;
+  static constexpr int kSmem = 1024 + kStages * kStage + kBar + kXbuf + kTok + kOst + kERec + 64;
   static_assert(kStages >= 3, "pipeline depth");
   static_assert(kBar <= 1024, "barrier area");
   static_assert(kSmem <= 227 * 1024 - 512, "shared memory");
@@ -157,6 +173,11 @@ __device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, 
       return false;
     }
   }
+}
+
+template <typename P>
+__device__ __forceinline__ P* u64ptr(uint32_t lo, uint32_t hi) {
+  return reinterpret_cast<P*>((static_cast<uint64_t>(hi) << 32) | lo);
 }
 
 // Byte offset of code k of token t in an input's tiled codes (k a multiple of 4).
@@ -465,6 +486,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   float* tsc = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(xbuf) + C::kXbuf);
   int32_t* trs = reinterpret_cast<int32_t*>(tsc + 64);
   __half* ostage = reinterpret_cast<__half*>(trs + 64);
+  uint4* s_erec = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ostage) + C::kOst);
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_flag;
@@ -766,6 +788,20 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
     bool ok = true;
     int n = 0;
     int ui = u_begin;
+    // epilogue records of units [rec0, rec0 + kERecMax) staged in shared memory
+    const uint4* erecs = reinterpret_cast<const uint4*>(ws + H.off_erec);
+    int rec0 = u_begin;
+    auto stage_recs = [&](int u0) {
+      named_bar_sync(1, kPEpi);                // the previous records are no longer read
+      const int nq = 4 * min(kERecMax, u_end - u0);
+      for (int i = et; i < nq; i += kPEpi) s_erec[i] = __ldg(erecs + 4 * u0 + i);
+      named_bar_sync(1, kPEpi);
+      rec0 = u0;
+    };
+    if (u_begin < u_end) stage_recs(u_begin);
+    bool have_next = false;
+    float g_next = 0.0f, b_next = 0.0f;
+    int32_t rs_next = 0;
     for (int L = 0; L < H.n_levels; ++L) {
       // 1. quantise a share of this level's input rows (the 128 threads take one row at a time)
       const int ib = H.in_begin[L], ie = H.in_begin[L + 1];
@@ -798,15 +834,50 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
       named_bar_sync(1, kPEpi);
       if (!s_qflag) ok = false;
       // 2. this CTA's units of level L
-      while (ok && ui < u_end && projs[units[ui].proj].level == L) {
-        // plan records are copied into registers (output stores cannot alias them); the
-        // per-token scale and code sum are staged while the accumulator is still being built
-        const PUnit u = units[ui];
-        const PProj pj = projs[u.proj];
-        const PIn in = ins[pj.in];
+      while (ok && ui < u_end) {
+        if (ui >= rec0 + kERecMax) stage_recs(ui);
+        const uint4* rq = s_erec + 4 * (ui - rec0);
+        const uint4 q0 = rq[0], q1 = rq[1], q2 = rq[2], q3 = rq[3];
+        if (static_cast<int>(q3.z) != L) break;
+        // the unit's record, in registers (output stores cannot alias them)
+        struct {
+          int tile, nsplit, part_off, tile_id, nkb;
+        } u = {static_cast<int>(q2.x), static_cast<int>(q2.y), static_cast<int>(q2.z),
+               static_cast<int>(q2.w), static_cast<int>(q3.x)};
+        PProj pj = {};
+        pj.y = u64ptr<void>(q0.x, q0.y);
+        pj.N = static_cast<int32_t>(q3.y);
+        pj.glu = static_cast<int32_t>(q3.w & 1u);
+        pj.ydt = static_cast<int32_t>(q3.w >> 1);
+        // this unit's per-token scale and code sum (requested while the previous unit was
+        // finished, when that one was of the same level), then the next unit's
+        float gv = 0.0f, bv = 0.0f;
+        int32_t rv = 0;
+        if (have_next) {
+          gv = g_next;
+          rv = rs_next;
+          bv = b_next;
+        } else if (et < T) {
+          gv = __ldcg(u64ptr<const float>(q1.x, q1.y) + et);
+          rv = __ldcg(u64ptr<const int32_t>(q1.z, q1.w) + et);
+          bv = __ldg(u64ptr<const float>(q0.z, q0.w));
+        }
+        have_next = false;
+        if (ui + 1 < u_end && ui + 1 < rec0 + kERecMax) {
+          const uint4* rn = s_erec + 4 * (ui + 1 - rec0);
+          const uint4 n0 = rn[0], n1 = rn[1], n3 = rn[3];
+          if (static_cast<int>(n3.z) == L) {   // its codes exist (this level's barrier passed)
+            if (et < T) {
+              g_next = __ldcg(u64ptr<const float>(n1.x, n1.y) + et);
+              rs_next = __ldcg(u64ptr<const int32_t>(n1.z, n1.w) + et);
+              b_next = __ldg(u64ptr<const float>(n0.z, n0.w));
+            }
+            have_next = true;
+          }
+        }
         if (et < T) {
-          tsc[et] = __fmul_rn(__fdiv_rn(__ldcg(in.gamma + et), 127.0f), __ldg(pj.beta));
-          trs[et] = __ldcg(in.rowsum + et);
+          tsc[et] = __fmul_rn(__fdiv_rn(gv, 127.0f), bv);
+          trs[et] = rv;
         } else if (et < 64) {
           tsc[et] = 0.0f;   // padding tokens of the last chunk
           trs[et] = 0;
@@ -939,6 +1010,7 @@ struct Plan {
   std::vector<PIn> ins;
   std::vector<PProj> projs;
   std::vector<PUnit> units;
+  std::vector<PERec> erec;
   std::vector<int32_t> ctaoff;
   PHeader h;
   size_t bytes = 0;
@@ -1101,6 +1173,8 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
   off = al(off + P.projs.size() * sizeof(PProj), 256);
   h.off_units = static_cast<int64_t>(off);
   off = al(off + P.units.size() * sizeof(PUnit), 256);
+  h.off_erec = static_cast<int64_t>(off);
+  off = al(off + P.units.size() * sizeof(PERec), 256);
   h.off_ctaoff = static_cast<int64_t>(off);
   off = al(off + P.ctaoff.size() * sizeof(int32_t), 256);
   h.off_tilectr = static_cast<int64_t>(off);
@@ -1129,6 +1203,25 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
     off = al(off + static_cast<size_t>(q.N / 128) * q.nst * kPWStage, 256);
   }
   P.bytes = off;
+  P.erec.resize(P.units.size());
+  for (size_t i = 0; i < P.units.size(); ++i) {
+    const PUnit& u = P.units[i];
+    const PProj& q = P.projs[u.proj];
+    const PIn& in = P.ins[q.in];
+    PERec& e = P.erec[i];
+    e.y = q.y;
+    e.beta = q.beta;
+    e.gamma = in.gamma;
+    e.rowsum = in.rowsum;
+    e.tile = u.tile;
+    e.nsplit = u.nsplit;
+    e.part_off = u.part_off;
+    e.tile_id = u.tile_id;
+    e.nkb = u.nkb;
+    e.N = q.N;
+    e.level = q.level;
+    e.flags = (q.glu ? 1 : 0) | (q.ydt << 1);
+  }
   int k = 0;
   for (int L = 0; L <= n_levels; ++L) {
     while (k < static_cast<int>(P.ins.size()) && P.ins[k].level < L) ++k;
@@ -1222,6 +1315,7 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   std::memcpy(img.data() + P.h.off_in, P.ins.data(), P.ins.size() * sizeof(PIn));
   std::memcpy(img.data() + P.h.off_proj, P.projs.data(), P.projs.size() * sizeof(PProj));
   std::memcpy(img.data() + P.h.off_units, P.units.data(), P.units.size() * sizeof(PUnit));
+  std::memcpy(img.data() + P.h.off_erec, P.erec.data(), P.erec.size() * sizeof(PERec));
   std::memcpy(img.data() + P.h.off_ctaoff, P.ctaoff.data(), P.ctaoff.size() * sizeof(int32_t));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // pageable source: the copy has consumed the host buffer when cudaMemcpyAsync returns
