@@ -493,7 +493,8 @@ def run_gpu(args, rank, world, local_rank):
                     "peak": round(2 * bf16_peak, 1), "unit": "TOPS",
                     "frac": round(achieved / (2 * bf16_peak), 4),
                     "peak_source": peak_kind + " (2 x bf16 dense, the nominal int8/bf16 ratio)",
-                    "ops_per_launch": dom[3] / dom[1], "traffic": None}
+                    "ops_per_launch": dom[3] / dom[1],
+                    "traffic": profiled_traffic(dominant, wl.name)}
     else:
         achieved = dom[2] / dom_s / 1e9
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
