@@ -42,9 +42,9 @@
 namespace mmf {
 namespace {
 
-// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 and 10-13 unpack (even and odd stages),
-// 6-9 quantise + epilogue.
-constexpr int kPThreads = 448;
+// Warp roles: 0 TMA producer, 1 and 15 MMA issuers (even and odd stages; warp 1 alone for
+// 64-token tiles), 2-5 and 10-13 unpack (even and odd stages), 6-9 quantise + epilogue, 14 idle.
+constexpr int kPThreads = 512;
 constexpr int kPEpi = 128;
 constexpr int kPEpiT0 = 192;               // first epilogue thread
 constexpr int kPKB = 128;                  // K per TMEM slot (one sub-block)
@@ -444,8 +444,8 @@ __device__ __forceinline__ void store_tile(const PProj& pj, int tile, int T, int
   }
 }
 
-// Loads CH accumulator columns at taddr and, when `two`, adds the partial sum held 32 columns
-// further on.
+// Loads CH accumulator columns of the partial sums selected by `mask` (bit 0: at taddr, bit 1:
+// 32 columns further on) and adds them.
 template <int CH>
 __device__ __forceinline__ void load_acc(uint32_t taddr, int32_t (&v)[CH]) {
   uint32_t u[32];
@@ -461,9 +461,9 @@ __device__ __forceinline__ void load_acc(uint32_t taddr, int32_t (&v)[CH]) {
 }
 
 template <int CH>
-__device__ __forceinline__ void load_acc_sum(uint32_t taddr, bool two, int32_t (&v)[CH]) {
-  load_acc<CH>(taddr, v);
-  if (two) {
+__device__ __forceinline__ void load_acc_sum(uint32_t taddr, int mask, int32_t (&v)[CH]) {
+  load_acc<CH>(mask == 2 ? taddr + 32u : taddr, v);
+  if (mask == 3) {
     int32_t w[CH];
     load_acc<CH>(taddr + 32u, w);
 #pragma unroll
@@ -476,6 +476,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
 program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_ns) {
   using C = PCfg<BN>;
   constexpr int S = C::kStages;
+  // With BN <= 32 two MMA warps on different SM sub-partitions take alternate stages, each into
+  // its own partial accumulator (32 columns of the unit's 64); the epilogue adds the two.
+  constexpr bool kTwoMma = kSplitAcc<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -517,10 +520,10 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
     }
     for (int gi = 0; gi < kPGroups; ++gi) mbar_init(afull(gi), 4);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(accfull(b), 1);
+      mbar_init(accfull(b), kTwoMma ? 2 : 1);   // one commit per MMA warp
       mbar_init(accempty(b), 4);
     }
-    mbar_init(drainbar, 1);
+    mbar_init(drainbar, kTwoMma ? 2 : 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -637,8 +640,78 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         mbar_wait_bounded(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1),
                           kPDrainNs, nullptr, status);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (kTwoMma && (warp == 1 || warp == 15)) {
+    // ------------------------------------------------------------------ MMA issuers (BN <= 32)
+    // Warp 1 takes the even stages and warp 15 the odd ones; each adds its stages' MMAs into
+    // its own partial accumulator, columns 64b + 32 * mset.  A warp with no stage in a unit
+    // still commits to accfull(b) (after the accumulator is free), so that the epilogue always
+    // sees two arrivals per unit.
+    const int mset = warp == 1 ? 0 : 1;
+    constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
+    const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
+    uint32_t c = 0;                      // stage counter (32-bit: cheap % and /)
+    bool ok = true;
+    int n = 0;
+    int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
+    for (int ui = u_begin; ui < u_end && ok; ++ui, ++n) {
+      const int nkb = next_nkb;
+      if (ui + 1 < u_end) next_nkb = units[ui + 1].nkb;   // overlaps this unit's MMAs
+      const int b = n & 1;
+      const int ns = (nkb + kPSub - 1) / kPSub;
+      // this warp's stages of the unit are s = first_s, first_s + 2, ... <= last_s
+      const int first_s = static_cast<int>((c & 1) != static_cast<uint32_t>(mset));
+      const int last_s = ns - 1 - static_cast<int>(((c + ns - 1) & 1) != static_cast<uint32_t>(mset));
+      const uint32_t d = tmem + static_cast<uint32_t>(b * 64 + mset * 32);
+      if (n >= 2) {   // every MMA warp, even one with no stage here (see above)
+        const bool w = mbar_wait_bounded(accempty(b), static_cast<uint32_t>(((n >> 1) - 1) & 1),
+                                         limit_ns, abort_flag, status);
+        if (!__all_sync(0xFFFFFFFFu, w)) break;
+      }
+      if (first_s >= ns) {               // no stage of this warp in the unit
+        tc_fence_after();
+        tc_commit_warp(accfull(b));
+        c += static_cast<uint32_t>(ns);
+        continue;
+      }
+      for (int k = 0; k < nkb; k += kPSub, ++c) {
+        if ((c & 1) != static_cast<uint32_t>(mset)) continue;
+        const int nsub = min(kPSub, nkb - k);
+        const int st = static_cast<int>(c % S);
+        const int gi = static_cast<int>(c % kPGroups);
+        const bool w = mbar_wait_bounded(afull(gi), static_cast<uint32_t>((c / kPGroups) & 1),
+                                         limit_ns, abort_flag, status);
+        if (!__all_sync(0xFFFFFFFFu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int s_idx = k / kPSub;
+        const uint64_t bst = bdesc0 + static_cast<uint64_t>((st * C::kAct) >> 4);
+        const uint32_t ast = tmem + kPACol0 + gi * kPSub * 32;
+        auto sub = [&](int i) {
+          const uint64_t bd = bst + static_cast<uint64_t>((i * C::kActSub) >> 4);
+          const uint32_t ad = ast + i * 32;
+          tc_mma_i8_ts_warp(d, ad, bd, idesc, (s_idx == first_s && i == 0) ? 0u : 1u);
+          tc_mma_i8_ts_warp(d, ad + 8, bd + 2, idesc, 1u);
+          tc_mma_i8_ts_warp(d, ad + 16, bd + 4, idesc, 1u);
+          tc_mma_i8_ts_warp(d, ad + 24, bd + 6, idesc, 1u);
+        };
+        if (nsub == kPSub) {
+#pragma unroll
+          for (int i = 0; i < kPSub; ++i) sub(i);
+        } else {
+          for (int i = 0; i < nsub; ++i) sub(i);
+        }
+        tc_commit_warp(empty(st));
+        if (s_idx == last_s) tc_commit_warp(accfull(b));
+      }
+    }
+    // Drain: nothing this warp issued may still be running when TMEM is freed.
+    tc_commit_warp(drainbar);
+    mbar_wait_bounded(drainbar, 0u, kPDrainNs, nullptr, status);
+    __syncwarp();
+  } else if (!kTwoMma && warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (BN = 64)
     // The whole warp runs the loop (waits and their outcomes are warp-uniform) and one elected
     // lane issues each MMA and commit.
     constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
@@ -704,7 +777,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
     tc_commit_warp(drainbar);
     mbar_wait_bounded(drainbar, 0u, kPDrainNs, nullptr, status);
     __syncwarp();
-  } else if (warp < 6 || warp >= 10) {
+  } else if (warp < 6 || (warp >= 10 && warp < 14)) {
     // ------------------------------------------------------------------ unpack
     // Each lane owns one tile row (= TMEM lane): per stage it reads its row's 128-byte weight
     // line once and unpacks its sub-blocks (32 bytes, 128 codes each) into TMEM slots.  Two
@@ -778,7 +851,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         if (lane == 0) mbar_arrive(afull(gi));
       }
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------------------------ quantise + epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;
@@ -787,6 +860,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
     constexpr int CH = C::kCh;
     bool ok = true;
     int n = 0;
+    uint32_t cs = 0;                     // stage counter (the MMA warps' c)
     int ui = u_begin;
     // epilogue records of units [rec0, rec0 + kERecMax) staged in shared memory
     const uint4* erecs = reinterpret_cast<const uint4*>(ws + H.off_erec);
@@ -889,12 +963,16 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
         if (!ok) break;
         tc_fence_after();
         const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(b * 64);
-        const bool two = kSplitAcc<BN> && u.nkb > 1;   // the odd-sub-block partial exists
+        // partial accumulators written for this unit: one per MMA warp (stage parity), both
+        // when the unit has two or more stages
+        const int ns_u = (u.nkb + kPSub - 1) / kPSub;
+        const int pmask = !kTwoMma ? 1 : (ns_u >= 2 ? 3 : 1 << static_cast<int>(cs & 1));
+        cs += static_cast<uint32_t>(ns_u);
         if (u.nsplit == 1) {
 #pragma unroll 1
           for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
             int32_t v[CH];
-            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), two, v);
+            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), pmask, v);
             finalize_chunk<CH>(pj, u.tile, T, c0, v, r, tsc, trs, xbuf, ostage);
           }
           tc_fence_before();
@@ -910,7 +988,7 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
 #pragma unroll 1
           for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
             int32_t v[CH];
-            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), two, v);
+            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), pmask, v);
 #pragma unroll
             for (int jj = 0; jj < CH; ++jj) atomicAdd(tacc + (c0 + jj) * 128 + r, v[jj]);
           }
