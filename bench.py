@@ -100,27 +100,35 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_sha():
+# the sources each profiled kernel is built from (its own file plus the shared device headers)
+KERNEL_SOURCES = {
+    "program_kernel": ["program.cu"],
+    "ternary_gemm": ["ternary_gemm.cu"],
+    "act_quant": ["act_quant.cu"],
+}
+
+
+def kernel_source_sha(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ternary_weight_lm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in sorted(KERNEL_SOURCES[kernel] + ["kernels.cuh", "ptx.cuh"]):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel, workload):
-    """dram bytes per launch recorded from an ncu capture in profiles/, if the kernel sources
-    are unchanged since (the summary names the source hash it was taken at)."""
+    """dram bytes per launch recorded from an ncu capture in profiles/, if the kernel's sources
+    are unchanged since (the summary names the hash of those sources it was taken at)."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path, encoding="utf-8").read()
     m_sha = re.search(r"source_sha:\s*([0-9a-f]+)", text)
     m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_sha or not m_b or m_sha.group(1) != kernel_source_sha():
+    if kernel not in KERNEL_SOURCES or not m_sha or not m_b or \
+            m_sha.group(1) != kernel_source_sha(kernel):
         return None
     return float(m_b.group(1))
 
