@@ -110,3 +110,38 @@ def test_program_fp32_inputs_with_norm_weights():
         y_ref = oracle_forward_from_parts(x, Wp.cpu().numpy(), float(beta.item()), spec.K,
                                           g=g, glu=spec.glu)
         assert_out_close(p["y"].double().cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("T", [1, 2, 8, 16, 17, 32, 33, 64])
+def test_program_short_rows_and_partial_stages(T):
+    """Projections whose units have a single stage (K <= 512), a partial last stage (K not a
+    multiple of 512) and several levels, at every token-tile size and its boundaries.  With
+    16- and 32-token tiles the MMA warps take alternate stages, so a unit of one stage leaves
+    one of them without work: its partial must not be added."""
+    shapes = [(128, 256, False, 0), (384, 128, False, 0), (512, 384, True, 0),
+              (640, 256, False, 1), (1152, 128, False, 1), (896, 512, True, 2)]
+    projs, host = [], []
+    xs = {}
+    for i, (K, N, glu, level) in enumerate(shapes):
+        if K not in xs:
+            xs[K] = to_dev(synth.activations(T + K, f"short/x{K}", T, K, dtype=np.float16))
+        W = synth.weights(40 + i, f"short/{i}", N, K)
+        Wp, beta = mmf.quantize_weights(to_dev(W))
+        y = torch.full((T, N // 2 if glu else N), float("nan"), dtype=torch.float16, device=DEV)
+        projs.append(dict(x=xs[K], norm_w=None, Wp=Wp, beta=beta, y=y, glu=glu, level=level))
+        host.append((K, glu, Wp, beta))
+    prog = mmf.Program(projs, T)
+    for rep in range(2):
+        for p in projs:
+            p["y"].fill_(float("nan"))
+        prog.run()
+        torch.cuda.synchronize()
+        assert mmf.mmf_get_device_status() == 0
+        ref = _reference_outputs([dict(p, y=torch.empty_like(p["y"])) for p in projs])
+        for i, p in enumerate(projs):
+            np.testing.assert_array_equal(p["y"].cpu().numpy(), ref[i].cpu().numpy(),
+                                          err_msg=f"projection {i} run {rep}")
+    for (K, glu, Wp, beta), p in zip(host, projs):
+        y_ref = oracle_forward_from_parts(p["x"].cpu().numpy(), Wp.cpu().numpy(),
+                                          float(beta.item()), K, glu=glu)
+        assert_out_close(p["y"].double().cpu().numpy(), y_ref)
