@@ -17,10 +17,11 @@
 //        producer thread streams the unit's packed weights (re-tiled at init into 16 KB
 //        blocks, one contiguous bulk copy per stage; ahead of time, across levels) and, once
 //        Q[L] has passed, the stage's activation codes (written tiled by step 1, one copy);
-//        four warps unpack the 2-bit codes into TMEM; a fifth issues tcgen05 kind::i8 MMAs into
-//        one of two TMEM accumulators; four more dequantise (and apply the GLU) or, for a tile
-//        split over several CTAs, add the int32 partial sums into the tile's accumulator, the
-//        last split finishing the tile;
+//        two sets of four warps unpack the 2-bit codes of alternate stages into TMEM; one or
+//        two warps issue tcgen05 kind::i8 MMAs into one of two TMEM accumulators; the four
+//        epilogue warps dequantise (and apply the GLU) or, for a tile split over several CTAs,
+//        add the int32 partial sums into the tile's accumulator, the last split finishing the
+//        tile;
 //     3. every CTA arrives on grid barrier O[L]; the next level may read this level's outputs.
 // Grid barriers are counters in the workspace with bounded waits; a timeout anywhere sets a
 // poison flag that makes every other wait give up too, and is reported as MMF_ERR_TIMEOUT.
