@@ -8,11 +8,16 @@ epilogue (x_mlp) and down_proj fed by gate_proj's GLU output h.  The default dat
 layer's other inputs come from the recurrence, the residual stream and the norms, which are
 outside the path, so they are seeded synthetic activations, one set per layer.  "--dataflow
 chained" instead feeds every projection from an earlier one (o from g, gate from o, the next
-layer from down), the dependency depth of a real layer-by-layer decode.  Each projection is the full
-forward: RMSNorm + int8 activation quantisation, then the tcgen05 ternary contraction with
-the dequantisation epilogue.  Weights are quantised and packed once before timing (the
-offline step of the method); packed weights rotate over enough distinct copies that every
-step streams them from HBM, not L2.
+layer from down), the dependency depth of a real layer-by-layer decode.  Each projection is the
+full forward: RMSNorm + int8 activation quantisation, then the tcgen05 ternary contraction with
+the dequantisation epilogue; projections that read the same input (i/f/g) share its
+quantisation.  Weights are quantised and packed once before timing (the offline step of the
+method); packed weights rotate over enough distinct copies that every step streams them from
+HBM, not L2.
+
+The headline line times the largest single-GPU workload (the 1.3B-shaped prefill, tensor-bound)
+and, in a "decode" object beside it, the HBM-bound decode workloads (1.3B at 1/8/64 tokens,
+2.7B at 8 tokens), each with its own step time, weight GB/s, roofline fraction and clocks.
 
 Arms:
   default            the CUDA library through its C ABI; the timed region replays CUDA
@@ -24,9 +29,12 @@ torch.distributed.run, one replica per GPU (the projection shards by tokens with
 exchange), timing = max over ranks.  Rank 0 prints one JSON line.
 """
 import argparse
+import concurrent.futures
 import hashlib
 import json
+import math
 import os
+import platform
 import re
 import statistics
 import subprocess
@@ -46,21 +54,29 @@ METRIC = "FusedBitLinear tokens/s; weight GB/s (decode), int8 TOPS (prefill) vs 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_INT8_TOPS = 4500.0          # B200 dense int8, datasheet
+INT8_PER_BF16 = 2.0                 # nominal dense int8 / bf16 throughput ratio
+GRAPH_SAMPLES = 8                   # distinct step graphs carrying per-launch timing events
 
 
 # ----------------------------------------------------------------------------- helpers
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mmf", "reference"], default="mmf")
     ap.add_argument("--workload", default=synth.workloads.DEFAULT,
                     choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--decode", default=",".join(synth.workloads.DECODE_SUITE),
+                    help="comma-separated decode workloads reported beside the headline "
+                         "('' for none)")
+    ap.add_argument("--decode-seconds", type=float, default=0.5,
+                    help="least timed GPU time of each decode entry")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="target host time of the CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="target host time of each CPU-baseline leg")
     ap.add_argument("--path", choices=["auto", "program", "launches"], default="auto",
                     help="one program launch per step (decode, T <= 64) or per-projection launches")
     ap.add_argument("--dataflow", choices=sorted(DATAFLOWS), default="path",
@@ -91,13 +107,26 @@ def aggregate_throughput(tokens_per_step, steps, world, max_seconds):
 
 
 def measured_peaks():
+    """(hbm GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
     except Exception:
-        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def tensor_peak(clocks, bf16_burst, bf16_sustained):
+    """int8 peak for a kernel timed in the headline's long loop: the measured bf16 dense rate
+    times the nominal int8/bf16 ratio, burst while the SM clock stayed near its maximum, the
+    sustained (power-capped) figure when it did not."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    throttled = sm is not None and mx and sm < 0.95 * mx
+    if throttled:
+        return INT8_PER_BF16 * bf16_sustained, "sustained"
+    return INT8_PER_BF16 * bf16_burst, "burst"
 
 
 # the sources each profiled kernel is built from (its own file plus the shared device headers)
@@ -171,24 +200,30 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, flag in zip(names, parts[5:9]):
-                if flag.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return summarise_clock_lines(self.lines)
+
+
+def summarise_clock_lines(lines):
+    """Median SM clock, the maximum, and every throttle reason seen active, from nvidia-smi
+    csv lines (index, sm, max sm, power, active mask, four reason flags)."""
+    sm, mx, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            mx = float(parts[2])
+        except ValueError:
+            continue
+        for name, flag in zip(names, parts[5:9]):
+            if flag.lower() == "active":
+                reasons.add(name)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+            "samples": len(sm)}
 
 
 # ----------------------------------------------------------------------------- workload
@@ -199,9 +234,9 @@ def projection_bytes(p, T):
     return p.N * p.K // 4 + T * p.K + 8 * T + 2 * T * n_out
 
 
-def quant_bytes(p, T, in_bytes=2):
+def quant_bytes(K, T, in_bytes=2):
     """Algorithmic bytes of one RMSNorm + quantisation launch: x in, codes + gamma + sums out."""
-    return in_bytes * T * p.K + T * p.K + 8 * T
+    return in_bytes * T * K + T * K + 8 * T
 
 
 def step_bytes(wl):
@@ -243,7 +278,7 @@ DATAFLOW_TEXT = {
 
 
 class GpuWorkload:
-    """Device buffers for one replica: packed weight copies, the step input, per-layer outputs,
+    """Device buffers for one replica: packed weight copies, the step inputs, the step outputs,
     and either one planned program per weight copy (T <= 64) or per-projection launches."""
 
     def __init__(self, wl, device, path="auto", dataflow="path"):
@@ -262,18 +297,23 @@ class GpuWorkload:
         # one seeded layer quantised by the library; every other layer and copy is a byte copy at
         # a distinct address (identical bytes stream exactly like distinct ones)
         self.Wp, self.beta = {}, {}
+        nz = 0
         for p in wl.projections:
             W = torch.from_numpy(synth.weights(0, p.name, p.N, p.K)).to(device)
             Wp0, b0 = mmf.quantize_weights(W)
             del W
+            # nonzero codes of this projection (2-bit fields holding e = c + 1 != 1), counted
+            # on the side for the report; the step itself never looks at this
+            nz += sum(int(((Wp0 >> s) & 3).ne(1).sum()) for s in (0, 2, 4, 6))
             n = self.copies * wl.layers
             self.Wp[p.name] = [Wp0] + [Wp0.clone() for _ in range(n - 1)]
             self.beta[p.name] = [b0] + [b0.clone() for _ in range(n - 1)]
+        self.nonzero_frac = nz / wl.weights_per_layer
         # step inputs: "path" has one set of synthetic activations per layer and source,
-        # "chained" only the first layer's input
+        # "chained" only the first layer's input.  All of a step's outside inputs are views of
+        # one contiguous device buffer, and all of its outputs views of another, so that the
+        # end-to-end measurement moves each with one copy per step.
         srcs = sorted({SOURCE_OF.get(p.name, "x_attn") for p in wl.projections} - {"h"})
-        # all of a step's outside inputs are views of one contiguous device buffer, so that the
-        # end-to-end measurement brings them in with one host-to-device copy per step
         nl = wl.layers if dataflow == "path" else 1
         srcs_l = srcs if dataflow == "path" else ["x_attn"]
         self.xin_buf = torch.empty((nl * len(srcs_l), T, H),
@@ -290,9 +330,15 @@ class GpuWorkload:
                 d[src] = v
             self.xin.append(d)
         self.x = self.xin[0]["x_attn"]
-        self.y = [{p.name: torch.empty((T, p.N // 2 if p.glu else p.N), dtype=self.ydt,
-                                       device=device) for p in wl.projections}
-                  for _ in range(wl.layers)]
+        widths = [p.N // 2 if p.glu else p.N for p in wl.projections]
+        self.yout_buf = torch.empty(wl.layers * T * sum(widths), dtype=self.ydt, device=device)
+        self.y, off = [], 0
+        for _ in range(wl.layers):
+            d = {}
+            for p, w in zip(wl.projections, widths):
+                d[p.name] = self.yout_buf[off:off + T * w].view(T, w)
+                off += T * w
+            self.y.append(d)
         self.use_program = (path == "program") or (path == "auto" and T <= 64)
         self.programs = []
         if self.use_program:
@@ -300,8 +346,6 @@ class GpuWorkload:
                 self.programs.append(mmf.Program(self.projection_list(c), T))
         else:
             kmax = max(p.K for p in wl.projections)
-            nmax = max(p.N for p in wl.projections)
-            self.ws = mmf.workspace(mmf.mmf_forward_workspace_bytes(T, kmax, nmax), device)
             self.A = torch.empty((T, kmax), dtype=torch.int8, device=device)
             self.gamma = torch.empty(T, dtype=torch.float32, device=device)
             self.rowsum = torch.empty(T, dtype=torch.int32, device=device)
@@ -320,9 +364,13 @@ class GpuWorkload:
 
     @property
     def step_inputs(self):
-        """The device tensors a step reads from outside (copied in from the host in e2e): one
-        contiguous buffer holding every layer's inputs."""
-        return [self.xin_buf]
+        """The device tensor a step reads from outside (copied in from the host in e2e)."""
+        return self.xin_buf
+
+    @property
+    def step_outputs(self):
+        """The device tensor holding every output of a step (copied back in e2e)."""
+        return self.yout_buf
 
     def projection_list(self, c):
         out = []
@@ -335,112 +383,125 @@ class GpuWorkload:
                                 LEVELS_PER_LAYER["chained"] * l + self.level_of[p.name]))
         return out
 
-    @property
-    def final_output(self):
-        return self.y[-1]["down_proj" if "down_proj" in self.y[-1] else "proj"]
+    def launch_groups(self, l):
+        """The launches of layer l in dependency order: each distinct input is quantised once,
+        then every projection reading it runs its contraction."""
+        groups = []
+        for p in sorted(self.wl.projections, key=lambda q: self.level_of[q.name]):
+            x = self.input_of(l, p)
+            for gx, members in groups:
+                if gx is x:
+                    members.append(p)
+                    break
+            else:
+                groups.append((x, [p]))
+        return groups
 
-    def run_step(self, step_index):
-        """One step through the public entry points: one program launch, or two launches per
-        projection in dependency order."""
+    def run_step(self, step_index, mark=None):
+        """One step through the public entry points: one program launch, or per layer one
+        RMSNorm + quantisation launch per distinct input and one contraction launch per
+        projection.  `mark(kind, nbytes, nops)` is called after every launch (timing events)."""
         c = step_index % self.copies
         if self.use_program:
             self.programs[c].run()
+            if mark:
+                mark("program_kernel", step_bytes(self.wl), self.ops_per_step)
             return
-        mmf = self.mmf
+        mmf, T = self.mmf, self.wl.T
+        in_bytes = 4 if self.wl.x_dtype == "f32" else 2
         for l in range(self.wl.layers):
             li = c * self.wl.layers + l
-            for p in sorted(self.wl.projections, key=lambda q: self.level_of[q.name]):
-                f = mmf.mmf_bitlinear_glu_forward if p.glu else mmf.mmf_bitlinear_forward
-                f(self.input_of(l, p), None, 1e-8, self.Wp[p.name][li], self.beta[p.name][li],
-                  p.N, self.y[l][p.name], self.ws)
-
-    def run_step_timed(self, step_index, ev):
-        """The same step with every launch bracketed by CUDA events."""
-        torch, mmf = self.torch, self.mmf
-        c = step_index % self.copies
-        if self.use_program:
-            e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
-            e0.record()
-            self.programs[c].run()
-            e1.record()
-            ev.append(("program", step_bytes(self.wl), self.flops_per_step, e0, e1))
-            return
-        T = self.wl.T
-        for l in range(self.wl.layers):
-            li = c * self.wl.layers + l
-            for p in sorted(self.wl.projections, key=lambda q: self.level_of[q.name]):
-                A = self.A.view(-1)[:T * p.K].view(T, p.K)
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-                e0.record()
-                mmf.mmf_quantize_activations(self.input_of(l, p), None, 1e-8, A, self.gamma,
-                                             self.rowsum)
-                e1.record()
-                mmf.mmf_bitlinear_forward_quantized(A, self.gamma, self.rowsum,
-                                                    self.Wp[p.name][li], self.beta[p.name][li],
-                                                    p.N, p.glu, self.y[l][p.name])
-                e2.record()
-                ev.append(("act_quant", quant_bytes(p, T, 4 if self.wl.x_dtype == "f32" else 2),
-                           0, e0, e1))
-                ev.append(("ternary_gemm", projection_bytes(p, T), 2 * T * p.N * p.K, e1, e2))
+            for x, members in self.launch_groups(l):
+                K = x.shape[1]
+                A = self.A.view(-1)[:T * K].view(T, K)
+                mmf.mmf_quantize_activations(x, None, 1e-8, A, self.gamma, self.rowsum)
+                if mark:
+                    mark("act_quant", quant_bytes(K, T, in_bytes), 0)
+                for p in members:
+                    mmf.mmf_bitlinear_forward_quantized(A, self.gamma, self.rowsum,
+                                                        self.Wp[p.name][li],
+                                                        self.beta[p.name][li], p.N, p.glu,
+                                                        self.y[l][p.name])
+                    if mark:
+                        mark("ternary_gemm", projection_bytes(p, T), 2 * T * p.N * p.K)
 
     @property
     def launches_per_step(self):
-        return 1 if self.use_program else 2 * len(self.wl.projections) * self.wl.layers
+        if self.use_program:
+            return 1
+        return sum(1 + len(m) for m_l in range(self.wl.layers)
+                   for _, m in self.launch_groups(m_l))
 
     @property
     def packed_bytes_per_step(self):
         return self.wl.packed_bytes_per_layer * self.wl.layers
 
     @property
-    def flops_per_step(self):
+    def ops_per_step(self):
         return 2 * self.wl.T * self.wl.weights_per_layer * self.wl.layers
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_gpu(args, rank, world, local_rank):
+def gpu_index(local_rank):
+    if "CUDA_VISIBLE_DEVICES" in os.environ:
+        return os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]
+    return local_rank
+
+
+def time_workload(wl, args, dev, stream, world, local_rank, steps, warmup, with_e2e):
+    """Times `steps` steps of CUDA-graph replays of workload `wl`, inputs resident.  Per-kernel
+    durations come from timing events captured inside the same graphs (the launches path) or
+    are the step itself (the program path: one launch per step)."""
     import torch
     import ternary_weight_lm_b200 as mmf
-    from ternary_weight_lm_b200 import build as lib_build
-
-    if rank == 0:
-        lib_build.build()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device(f"cuda:{local_rank}")
-    wl = synth.WORKLOADS[args.workload]
     g = GpuWorkload(wl, dev, args.path, args.dataflow)
-    stream = torch.cuda.Stream(device=dev)
     T = wl.T
-
     with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
+        for i in range(max(warmup, 3)):
             g.run_step(i)
     torch.cuda.synchronize()
     if mmf.mmf_get_device_status() != 0:
         raise RuntimeError("device status reported a timeout during warm-up")
 
-    # CUDA graphs: one graph runs `chunk` consecutive steps (rotating the weight copies); the
-    # timed region replays it K // chunk times plus one graph for the remaining K % chunk steps
-    chunk = g.copies if g.use_program else 1
-    chunk = max(1, min(chunk, args.steps))
+    # ---- graphs.  Program path: one graph runs `chunk` consecutive steps (rotating the weight
+    # copies).  Launches path: GRAPH_SAMPLES graphs of one step each, with a timing event
+    # after every launch; the timed region replays them in turn.
+    records = []    # per sample graph: [(kind, nbytes, nops, ev_start, ev_end), ...]
 
-    def capture(n_steps):
+    def capture_program(n_steps):
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
             for i in range(n_steps):
                 g.run_step(i)
         return gr
 
-    with torch.cuda.stream(stream):
-        if g.use_program:
-            g_main = capture(chunk)
-            rem = args.steps % chunk
-            g_rem = capture(rem) if rem else None
-            graphs = None
-        else:
-            graphs = [capture_one(g, stream, j) for j in range(g.copies)]
+    def capture_timed(j):
+        gr = torch.cuda.CUDAGraph()
+        rec = []
+        with torch.cuda.graph(gr, stream=stream):
+            prev = torch.cuda.Event(enable_timing=True, external=True)
+            prev.record(stream)
+
+            def mark(kind, nbytes, nops):
+                nonlocal prev
+                e = torch.cuda.Event(enable_timing=True, external=True)
+                e.record(stream)
+                rec.append((kind, nbytes, nops, prev, e))
+                prev = e
+            g.run_step(j, mark)
+        records.append(rec)
+        return gr
+
+    if g.use_program:
+        chunk = max(1, min(g.copies, steps))
+        g_main = capture_program(chunk)
+        rem = steps % chunk
+        g_rem = capture_program(rem) if rem else None
+        graphs = None
+    else:
+        # one graph per weight copy (at least GRAPH_SAMPLES), so that the replays rotate over
+        # every copy
+        graphs = [capture_timed(j) for j in range(min(steps, max(GRAPH_SAMPLES, g.copies)))]
     torch.cuda.synchronize()
 
     def replay_steps(n):
@@ -448,13 +509,13 @@ def run_gpu(args, rank, world, local_rank):
             for _ in range(n // chunk):
                 g_main.replay()
             if n % chunk:
-                (g_rem if n % chunk == args.steps % chunk else capture(n % chunk)).replay()
+                g_rem.replay()
         else:
             for i in range(n):
-                graphs[i % g.copies].replay()
+                graphs[i % len(graphs)].replay()
 
     with torch.cuda.stream(stream):
-        replay_steps(max(args.warmup, 3) if not g.use_program else chunk)
+        replay_steps(chunk if g.use_program else len(graphs))
     torch.cuda.synchronize()
 
     def barrier():
@@ -462,15 +523,14 @@ def run_gpu(args, rank, world, local_rank):
             import torch.distributed as dist
             dist.barrier()
 
-    # ---- headline: K steps of graph replays, inputs resident in HBM
+    # ---- timed region: `steps` steps of graph replays
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else
-                      os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]) as clk:
+    with ClockSampler(gpu_index(local_rank)) as clk:
         barrier()
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             start.record()
-            replay_steps(args.steps)
+            replay_steps(steps)
             end.record()
         torch.cuda.synchronize()
         barrier()
@@ -478,60 +538,71 @@ def run_gpu(args, rank, world, local_rank):
     clocks = clk.summary()
     if mmf.mmf_get_device_status() != 0:
         raise RuntimeError("device status reported a timeout in the timed region")
-    value = aggregate_throughput(T, args.steps, world, elapsed_s)
-    ms_per_step = elapsed_s * 1e3 / args.steps
+    ms_per_step = elapsed_s * 1e3 / steps
 
-    # ---- instrumented pass: every launch bracketed by events (durations per kernel)
+    # ---- per-kernel durations inside the same replays
     per_kernel = {}
-    k_steps = min(args.steps, max(20, 2000 // max(1, g.launches_per_step)))
-    ev = []
-    with torch.cuda.stream(stream):
-        torch.cuda._sleep(int(1e9))     # let the host queue the whole pass before it runs
-        for i in range(k_steps):
-            g.run_step_timed(i, ev)
-    torch.cuda.synchronize()
-    for name, nbytes, nflops, e0, e1 in ev:
-        acc = per_kernel.setdefault(name, [0.0, 0, 0.0, 0.0])
-        acc[0] += e0.elapsed_time(e1)
-        acc[1] += 1
-        acc[2] += nbytes
-        acc[3] += nflops
+    if g.use_program:
+        per_kernel["program_kernel"] = [ms_per_step * steps, steps,
+                                        step_bytes(wl) * steps, g.ops_per_step * steps]
+        kernel_timing = ("one launch per step: the kernel's average is the step time of the "
+                         "timed graph replays")
+    else:
+        for rec in records:          # each sample graph's last replay inside the timed region
+            for kind, nbytes, nops, e0, e1 in rec:
+                acc = per_kernel.setdefault(kind, [0.0, 0, 0.0, 0.0])
+                acc[0] += e0.elapsed_time(e1)
+                acc[1] += 1
+                acc[2] += nbytes
+                acc[3] += nops
+        kernel_timing = (f"timing events captured between the launches of {len(graphs)} step "
+                         f"graphs, read after their last replay inside the timed region")
     total_ms = sum(v[0] for v in per_kernel.values())
-    kernels = {k: {"launches": v[1], "avg_us": 1e3 * v[0] / max(1, v[1]),
-                   "share": v[0] / total_ms if total_ms else None,
-                   "achieved_gbs": (v[2] / (v[0] / 1e3) / 1e9) if v[0] else None}
+    kernels = {k: {"launches": v[1], "avg_us": round(1e3 * v[0] / max(1, v[1]), 3),
+                   "share": round(v[0] / total_ms, 4) if total_ms else None,
+                   "achieved_gbs": round(v[2] / (v[0] / 1e3) / 1e9, 1) if v[0] else None,
+                   "achieved_tops": round(v[3] / (v[0] / 1e3) / 1e12, 1) if v[0] and v[3]
+                   else None}
                for k, v in per_kernel.items()}
     dominant = max(per_kernel, key=lambda k: per_kernel[k][0])
-    hbm_peak, bf16_peak, peak_kind = measured_peaks()
+    hbm_peak, bf16_burst, bf16_sust, peak_kind = measured_peaks()
     dom = per_kernel[dominant]
     dom_s = dom[0] / 1e3
-    if T > 64 and dom[3] > 0:
-        # prefill: the contraction is bound by the int8 tensor pipe; its peak is the measured
-        # bf16 GEMM throughput times the nominal int8/bf16 ratio (2)
+    if not g.use_program and dom[3] > 0 and T > 64:
+        # prefill: the contraction is bound by the int8 tensor pipe
         achieved = dom[3] / dom_s / 1e12
+        peak, which = tensor_peak(clocks, bf16_burst, bf16_sust)
+        step_tops = g.ops_per_step / (ms_per_step / 1e3) / 1e12
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1),
-                    "peak": round(2 * bf16_peak, 1), "unit": "TOPS",
-                    "frac": round(achieved / (2 * bf16_peak), 4),
-                    "peak_source": peak_kind + " (2 x bf16 dense, the nominal int8/bf16 ratio)",
+                    "peak": round(peak, 1), "unit": "TOPS", "frac": round(achieved / peak, 4),
+                    "peak_source": f"{peak_kind} bf16 dense ({which}) x {INT8_PER_BF16:g}, the "
+                                   f"nominal int8/bf16 ratio (no measured int8 entry)",
+                    "frac_of_burst_proxy": round(achieved / (INT8_PER_BF16 * bf16_burst), 4),
+                    "frac_of_sustained_proxy": round(achieved / (INT8_PER_BF16 * bf16_sust), 4),
+                    "frac_of_nominal_4p5_pops": round(achieved / NOMINAL_INT8_TOPS, 4),
+                    "step_tops": round(step_tops, 1),
+                    "step_frac": round(step_tops / peak, 4),
                     "ops_per_launch": dom[3] / dom[1],
+                    "nonzero_frac_of_weights": round(g.nonzero_frac, 4),
+                    "frac_counting_nonzero_adds_only": round(achieved * g.nonzero_frac / peak, 4),
                     "traffic": profiled_traffic(dominant, wl.name)}
     else:
         achieved = dom[2] / dom_s / 1e9
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1),
                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                    "peak_source": peak_kind,
+                    "peak_source": peak_kind + " copy bandwidth",
                     "bytes_per_launch": dom[2] / dom[1],
-                    "traffic": profiled_traffic("program_kernel" if dominant == "program"
-                                                else dominant, wl.name)}
+                    "traffic": profiled_traffic(dominant, wl.name)}
 
     # ---- e2e: the public API with host buffers, copies inside the timed region
     e2e = None
-    if not args.no_e2e:
-        hxs = [t.cpu().pin_memory() for t in g.step_inputs]
-        hy = torch.empty_like(g.final_output, device="cpu").pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in hxs)
+    if with_e2e:
+        hx = g.step_inputs.cpu().pin_memory()
+        hy = torch.empty_like(g.step_outputs, device="cpu").pin_memory()
+        h2d = hx.numel() * hx.element_size()
         d2h = hy.numel() * hy.element_size()
-        e2e_steps = min(args.steps, 200)
+        e2e_steps = max(3, min(steps, int(2.0 / max(1e-6, ms_per_step / 1e3 +
+                                                   (h2d + d2h) / 20e9))))
         with torch.cuda.stream(stream):
             for i in range(3):
                 g.run_step(i)
@@ -541,10 +612,9 @@ def run_gpu(args, rank, world, local_rank):
         with torch.cuda.stream(stream):
             s0.record()
             for i in range(e2e_steps):
-                for dst, src in zip(g.step_inputs, hxs):
-                    dst.copy_(src, non_blocking=True)
+                g.step_inputs.copy_(hx, non_blocking=True)
                 g.run_step(i)
-                hy.copy_(g.final_output, non_blocking=True)
+                hy.copy_(g.step_outputs, non_blocking=True)
             s1.record()
         torch.cuda.synchronize()
         barrier()
@@ -553,28 +623,70 @@ def run_gpu(args, rank, world, local_rank):
                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": e2e_steps,
                "path": ("mmf_program_run (one launch per step)" if g.use_program else
-                        "mmf_bitlinear_forward / _glu_forward per projection") +
-                       ", step inputs from pinned host memory, last output back to pinned host"}
+                        "mmf_quantize_activations once per distinct input + "
+                        "mmf_bitlinear_forward_quantized per projection") +
+                       ", every step input from pinned host memory in one copy, every step "
+                       "output back to pinned host memory in one copy"}
 
-    return {
-        "value": value, "ms_per_step": ms_per_step, "elapsed_s": elapsed_s, "clocks": clocks,
-        "roofline": roofline, "kernels": kernels, "e2e": e2e,
-        "launches": g.launches_per_step * args.steps,
-        "weight_gbs": g.packed_bytes_per_step * args.steps * world / elapsed_s / 1e9,
-        "int8_tops": g.flops_per_step * args.steps * world / elapsed_s / 1e12,
+    res = {
+        "workload": wl.name, "value": aggregate_throughput(T, steps, world, elapsed_s),
+        "ms_per_step": ms_per_step, "steps": steps, "clocks": clocks, "roofline": roofline,
+        "kernels": kernels, "kernel_timing": kernel_timing, "e2e": e2e,
+        "launches": g.launches_per_step * steps,
+        "weight_gbs": g.packed_bytes_per_step * steps * world / elapsed_s / 1e9,
+        "int8_tops": g.ops_per_step * steps * world / elapsed_s / 1e12,
         "copies": g.copies, "path": "program" if g.use_program else "launches",
     }
+    del g
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
 
-def capture_one(g, stream, j):
+def run_gpu(args, rank, world, local_rank):
     import torch
-    gr = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gr, stream=stream):
-        g.run_step(j)
-    return gr
+    from ternary_weight_lm_b200 import build as lib_build
+
+    if rank == 0:
+        lib_build.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device(f"cuda:{local_rank}")
+    stream = torch.cuda.Stream(device=dev)
+    wl = synth.WORKLOADS[args.workload]
+    head = time_workload(wl, args, dev, stream, world, local_rank, args.steps, args.warmup,
+                         not args.no_e2e)
+    decode = {}
+    for name in [n for n in args.decode.split(",") if n and n != args.workload]:
+        dwl = synth.WORKLOADS[name]
+        # each entry runs for at least --decode-seconds of GPU time (step times from 0.03 to
+        # 0.25 ms), so that the clock samples cover it
+        est_ms = max(0.02, dwl.packed_bytes_per_layer * dwl.layers / 3e12 * 1e3)
+        n_steps = max(args.steps, int(math.ceil(args.decode_seconds * 1e3 / est_ms)))
+        r = time_workload(dwl, args, dev, stream, world, local_rank, n_steps, args.warmup, False)
+        decode[name] = {k: r[k] for k in ("value", "ms_per_step", "steps", "clocks", "roofline",
+                                          "weight_gbs", "path", "launches", "copies")}
+        decode[name]["unit"] = "tokens/s"
+        decode[name]["tokens_per_step"] = dwl.T
+        decode[name]["layers_per_step"] = dwl.layers
+    head["decode"] = decode
+    return head
 
 
 # ----------------------------------------------------------------------------- oracle arm
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
 def oracle_sample(wl, n_tokens, dataflow="path"):
     """Inputs of a bounded sample of one step for the oracle: the first n_tokens tokens of the
     first layer's step inputs (the same seeded activations as the GPU arm's) and one layer's
@@ -583,9 +695,12 @@ def oracle_sample(wl, n_tokens, dataflow="path"):
     H = wl.projections[0].K
     xdt = np.float32 if wl.x_dtype == "f32" else np.float16
     srcs = sorted({SOURCE_OF.get(p.name, "x_attn") for p in wl.projections} - {"h"})
-    xs = {src: synth.activations(0, src, wl.T, H, dtype=xdt, outlier_frac=wl.outlier_frac,
-                                 outlier_scale=wl.outlier_scale)[:n_tokens]
-          for src in (srcs if dataflow == "path" else ["x_attn"])}
+    xs = {}
+    for src in (srcs if dataflow == "path" else ["x_attn"]):
+        x = synth.activations(0, src, wl.T, H, dtype=xdt, outlier_frac=wl.outlier_frac,
+                              outlier_scale=wl.outlier_scale)
+        xs[src] = np.ascontiguousarray(x[:n_tokens])
+        del x
     weights = {}
     for p in wl.projections:
         W = synth.weights(0, p.name, p.N, p.K)
@@ -594,13 +709,15 @@ def oracle_sample(wl, n_tokens, dataflow="path"):
     return xs, weights
 
 
-def oracle_step(wl, xs, weights, dataflow="path"):
+def oracle_step(wl, xs, weights, dataflow="path", pool=None, nthreads=1):
     """One layer of the step in the same data flow as the GPU arm, outputs rounded to the output
-    dtype where they feed the next projection."""
+    dtype where they feed the next projection.  With a thread pool, each projection's output
+    rows (weight rows) are split over `nthreads` threads, each running the oracle's own
+    accumulation on its rows (the oracle's C code runs without the interpreter lock)."""
     import oracle
     ydt = np.float32 if wl.y_dtype == "f32" else np.float16
     level_of = DATAFLOWS[dataflow]
-    outs = {}
+    outs, quant = {}, {}
     for p in sorted(wl.projections, key=lambda q: level_of[q.name]):
         if p.name == "down_proj":
             xin = outs["gate_proj"]
@@ -613,34 +730,72 @@ def oracle_step(wl, xs, weights, dataflow="path"):
         else:
             xin = outs["o_proj"]
         c, beta = weights[p.name]
-        q, gamma, _ = oracle.rmsnorm_actquant(xin)
-        y = oracle.dequant(oracle.ternary_accumulate(q, c), gamma, beta)
+        key = id(xin)
+        if key not in quant:
+            quant[key] = oracle.rmsnorm_actquant(xin)
+        q, gamma, _ = quant[key]
+        if pool is None or nthreads <= 1:
+            acc = oracle.ternary_accumulate(q, c)
+        else:
+            bounds = np.linspace(0, c.shape[0], nthreads + 1).astype(int)
+            parts = list(pool.map(lambda ab: oracle.ternary_accumulate(q, c[ab[0]:ab[1]]),
+                                  [(bounds[i], bounds[i + 1]) for i in range(nthreads)
+                                   if bounds[i + 1] > bounds[i]]))
+            acc = np.concatenate(parts, axis=1)
+        y = oracle.dequant(acc, gamma, beta)
         if p.glu:
             y = oracle.silu_glu(y)
         outs[p.name] = y.astype(ydt)
     return outs
 
 
-def oracle_tokens_per_s(wl, seconds, n_tokens=None, dataflow="path"):
-    """Time the oracle on bounded samples for about `seconds` of host time."""
-    if n_tokens is None:
-        n_tokens = min(wl.T, 8)
-    xs, weights = oracle_sample(wl, n_tokens, dataflow)
-    oracle_step(wl, xs, weights, dataflow)       # warm
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle_step(wl, xs, weights, dataflow)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
+def _time_oracle(wl, xs, weights, n_tokens, seconds, dataflow, nthreads):
+    xs = {k: np.ascontiguousarray(v[:n_tokens]) for k, v in xs.items()}
+    pool = concurrent.futures.ThreadPoolExecutor(nthreads) if nthreads > 1 else None
+    try:
+        oracle_step(wl, xs, weights, dataflow, pool, nthreads)       # warm
+        reps, t0 = 0, time.perf_counter()
+        while True:
+            oracle_step(wl, xs, weights, dataflow, pool, nthreads)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    finally:
+        if pool is not None:
+            pool.shutdown()
     # one sample step covers one layer; a full step streams wl.layers layers
-    tps = n_tokens * reps / el / wl.layers
-    return tps, {"kind": "oracle", "cores": 1,
-                 "sample": f"first {n_tokens} of {wl.T} tokens through all "
-                           f"{len(wl.projections)} projections of one layer ({dataflow} data flow), repeated "
-                           f"{reps} times ({el:.1f} s); tokens/s scaled by 1/{wl.layers} "
-                           f"layers", "value": round(tps, 3), "unit": "tokens/s"}
+    return n_tokens * reps / el / wl.layers, reps, el
+
+
+def oracle_tokens_per_s(wl, seconds, dataflow="path", threads=None):
+    """The oracle on bounded samples of the step: one host thread, and all host cores with the
+    output rows of each projection split over threads.  Token counts are sized so that each
+    leg runs about `seconds`; prefill-sized steps use a slice of their tokens (at most 256),
+    marked as extrapolated."""
+    threads = threads or max(1, min(os.cpu_count() or 1, 64))
+    xs, weights = oracle_sample(wl, min(wl.T, 256), dataflow)
+    # the cost of one token through one layer, single-threaded
+    t1, _, _ = _time_oracle(wl, xs, weights, 1, 0.0, dataflow, 1)
+    per_tok = 1.0 / max(t1 * wl.layers, 1e-9)
+    n_single = int(max(1, min(wl.T, 256, seconds / per_tok / 2)))
+    n_thr = int(max(1, min(wl.T, 256, seconds * threads / per_tok / 2)))
+    v1, r1, el1 = _time_oracle(wl, xs, weights, n_single, seconds, dataflow, 1)
+    vt, rt, elt = _time_oracle(wl, xs, weights, n_thr, seconds, dataflow, threads)
+
+    def leg(v, n, reps, el, th):
+        return {"value": round(v, 3), "unit": "tokens/s", "threads": th,
+                "sample": f"first {n} of {wl.T} tokens through all {len(wl.projections)} "
+                          f"projections of one layer ({dataflow} data flow), repeated {reps} "
+                          f"times ({el:.1f} s); tokens/s scaled by 1/{wl.layers} layers",
+                "extrapolated": n < wl.T}
+    single = leg(v1, n_single, r1, el1, 1)
+    threaded = leg(vt, n_thr, rt, elt, threads)
+    return vt, {"kind": "oracle", "value": round(vt, 3), "unit": "tokens/s", "cores": threads,
+                "sample": threaded["sample"] + (" (extrapolated from the slice)"
+                                                if threaded["extrapolated"] else ""),
+                "single": single, "threaded": threaded,
+                "hardware_concurrency": os.cpu_count(), "cpu_model": cpu_model()}
 
 
 def run_reference(args, rank, world):
@@ -649,43 +804,54 @@ def run_reference(args, rank, world):
         return None
     # size each step so that warm-up + K steps stay within about two minutes
     df = args.dataflow
-    xs, weights = oracle_sample(wl, 1, df)
-    t0 = time.perf_counter()
-    oracle_step(wl, xs, weights, df)
-    per_token_layer = time.perf_counter() - t0
-    n_tok = int(max(1, min(wl.T, 120.0 / max(1, args.steps + args.warmup) / per_token_layer)))
-    xs, weights = oracle_sample(wl, n_tok, df)
-    for _ in range(args.warmup):
-        oracle_step(wl, xs, weights, df)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(wl, xs, weights, df)
-    el = time.perf_counter() - t0
+    threads = max(1, min(os.cpu_count() or 1, 64))
+    pool = concurrent.futures.ThreadPoolExecutor(threads) if threads > 1 else None
+    try:
+        xs, weights = oracle_sample(wl, 1, df)
+        t0 = time.perf_counter()
+        oracle_step(wl, xs, weights, df, pool, threads)
+        per_token_layer = time.perf_counter() - t0
+        n_tok = int(max(1, min(wl.T, 256,
+                               120.0 / max(1, args.steps + args.warmup) / per_token_layer)))
+        xs, weights = oracle_sample(wl, n_tok, df)
+        for _ in range(args.warmup):
+            oracle_step(wl, xs, weights, df, pool, threads)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_step(wl, xs, weights, df, pool, threads)
+        el = time.perf_counter() - t0
+    finally:
+        if pool is not None:
+            pool.shutdown()
     tps = n_tok * args.steps / el / wl.layers
-    cpu = {"kind": "oracle", "cores": 1, "value": round(tps, 3), "unit": "tokens/s",
+    cpu = {"kind": "oracle", "cores": threads, "value": round(tps, 3), "unit": "tokens/s",
            "sample": f"each step: first {n_tok} of {wl.T} tokens through every projection of "
-                     f"one layer; tokens/s scaled by 1/{wl.layers} layers"}
+                     f"one layer, output rows split over {threads} threads; tokens/s scaled by "
+                     f"1/{wl.layers} layers" + (" (extrapolated)" if n_tok < wl.T else ""),
+           "hardware_concurrency": os.cpu_count(), "cpu_model": cpu_model()}
     return {"impl": "reference", "metric": METRIC, "value": round(tps, 3), "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": config_of(wl, None, df), "cpu_baseline": cpu,
+            "config": config_of(wl, df), "cpu_baseline": cpu,
             "e2e": {"value": round(tps, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
-def config_of(wl, res, dataflow="path"):
-    c = {"workload": wl.name, "tokens_per_step": wl.T, "layers_per_step": wl.layers,
-         "projections": ",".join(p.name + ("(glu)" if p.glu else "") for p in wl.projections),
-         "x_dtype": wl.x_dtype, "y_dtype": wl.y_dtype, "parallelism": "replicas",
-         "dataflow": DATAFLOW_TEXT[dataflow]}
-    if res is not None:
-        c["weight_copies"] = res["copies"]
-        c["l2"] = ("packed weights rotate over %d distinct copies (%.0f MB > 2x L2); "
-                   "activations stay L2-resident as in a layer-by-layer decode"
-                   % (res["copies"], res["copies"] * wl.packed_bytes_per_layer * wl.layers / 1e6))
-        c["timing"] = "CUDA graph replays of whole steps, CUDA events on the launch stream"
-    return c
+def config_of(wl, dataflow="path"):
+    return {"workload": wl.name, "tokens_per_step": wl.T, "layers_per_step": wl.layers,
+            "projections": ",".join(p.name + ("(glu)" if p.glu else "") for p in wl.projections),
+            "x_dtype": wl.x_dtype, "y_dtype": wl.y_dtype, "parallelism": "replicas",
+            "dataflow": DATAFLOW_TEXT[dataflow]}
+
+
+def timing_setup(wl, res):
+    return {"weight_copies": res["copies"],
+            "l2": ("packed weights rotate over %d distinct copies (%.0f MB > 2x L2); "
+                   "activations as a layer-by-layer step leaves them"
+                   % (res["copies"], res["copies"] * wl.packed_bytes_per_layer * wl.layers / 1e6)),
+            "timing": "CUDA graph replays of whole steps, CUDA events on the launch stream",
+            "kernel_timing": res["kernel_timing"]}
 
 
 # ----------------------------------------------------------------------------- main
@@ -713,17 +879,18 @@ def main(argv=None):
                     "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                     "ms_per_step": round(res["ms_per_step"], 6), "higher_is_better": True,
                     "scaling": "weak", "vs_baseline": None, "dtype": "int8",
-                    "data": "synthetic", "config": config_of(wl, res, args.dataflow),
+                    "data": "synthetic", "config": config_of(wl, args.dataflow),
+                    "timing_setup": timing_setup(wl, res),
                     "weight_gbs": round(res["weight_gbs"], 1),
                     "int8_tops": round(res["int8_tops"], 2),
                     "path": res["path"],
                     "roofline": res["roofline"], "kernels": res["kernels"],
                     "clocks": res["clocks"], "e2e": res["e2e"],
                     "gpu_launches": res["launches"],
+                    "decode": res["decode"],
                 }
                 if not args.no_cpu_baseline and world == 1:
-                    _, cpu = oracle_tokens_per_s(wl, args.cpu_seconds,
-                                                 dataflow=args.dataflow)
+                    _, cpu = oracle_tokens_per_s(wl, args.cpu_seconds, dataflow=args.dataflow)
                     line["cpu_baseline"] = cpu
                 else:
                     line["cpu_baseline"] = None

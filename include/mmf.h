@@ -69,7 +69,9 @@ typedef enum {
   MMF_ERR_ALIGNMENT = 3,          /* a pointer not aligned as required */
   MMF_ERR_CUDA = 4,               /* a CUDA runtime or driver call failed */
   MMF_ERR_TIMEOUT = 5,            /* a device-side wait ran past its limit */
-  MMF_ERR_WORKSPACE = 6           /* workspace missing or smaller than required */
+  MMF_ERR_WORKSPACE = 6,          /* workspace missing or smaller than required */
+  MMF_ERR_RESOURCES = 7,          /* the device cannot hold every CTA of a program at once */
+  MMF_ERR_PLAN = 8                /* a program run found no valid plan in its workspace */
 } mmf_status;
 
 typedef enum { MMF_F32 = 0, MMF_F16 = 1 } mmf_dtype;
@@ -166,19 +168,31 @@ size_t mmf_program_workspace_bytes(const mmf_projection* p, int n, int64_t T);
  * groups projections that share an input into one quantisation, splits every level's
  * k-blocks over the SMs and zeroes the counters.  It also re-tiles every projection's packed
  * weights (Wp, canonical layout L1) into the workspace, in blocks that one contiguous copy
- * brings on chip: runs read that copy, so Wp may be freed after the init has executed, and a
- * change of the weights needs a new init.  The other pointers in `p` are baked into the plan:
- * every later mmf_program_run reads and writes those same buffers.  All work is
- * stream-ordered on `stream`.  1 <= T <= 64. */
+ * brings on chip: runs read that copy, so Wp may be freed once the init has executed (the
+ * program then holds one copy of the weights, not two), and a change of the weights needs a
+ * new init.  The other pointers in `p` are baked into the plan: every later mmf_program_run
+ * reads and writes those same buffers.  All device work is stream-ordered on `stream`; the
+ * init copies from pageable host memory, so it must not be captured into a CUDA graph.
+ * 1 <= T <= 64.  Returns MMF_ERR_RESOURCES if the device cannot hold one CTA on every SM at
+ * once (the runs' grid-wide waits need every CTA resident). */
 mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T, float eps, void* ws,
                             size_t ws_bytes, void* stream);
 
 /* Runs a planned program: one persistent launch, one CTA per SM.  Level by level, every CTA
  * quantises a share of the level's input rows (RMSNorm + int8), then streams its share of the
  * packed weights through the tcgen05 contraction (weights are prefetched across levels), and
- * the level ends when every output is written.  Grid-wide waits are bounded: on a timeout the
- * kernel records MMF_ERR_TIMEOUT (mmf_get_device_status) and returns; call mmf_program_init
- * again before the next run in that case.  Calls on one workspace must not overlap. */
+ * the level ends when every output is written.
+ * Co-residency: the CTAs wait for one another at every level, so the launch is made
+ * cooperative where the driver accepts that (it then places the whole grid at once, or fails
+ * with MMF_ERR_RESOURCES); where it does not, a run needs the whole GPU to itself.  Either way
+ * every grid-wide wait is bounded: a CTA that is never placed makes the others record
+ * MMF_ERR_TIMEOUT (mmf_get_device_status) and return instead of hanging; call
+ * mmf_program_init again before the next run in that case.
+ * The launch checks the plan in `ws` (a magic number, the init's generation, the token tile
+ * and the grid size): a workspace that no longer holds the plan it was initialised with is
+ * refused without any other read or write, and mmf_get_device_status then returns
+ * MMF_ERR_PLAN.  `ws` not passed to a successful mmf_program_init: MMF_ERR_INVALID_ARG.
+ * Calls on one workspace must not overlap. */
 mmf_status mmf_program_run(void* ws, void* stream);
 
 /* ---- forward without any allocation ------------------------------------------------------ */
@@ -203,7 +217,8 @@ mmf_status mmf_bitlinear_forward_noalloc(const void* x, mmf_dtype xdt, int64_t T
 /* ---- status ------------------------------------------------------------------------------ */
 
 /* Reads and clears the device status word of the current device (synchronises the device).
- * Returns MMF_OK, MMF_ERR_TIMEOUT if a kernel gave up on a wait since the last read, or
+ * Returns MMF_OK, MMF_ERR_TIMEOUT if a kernel gave up on a wait since the last read,
+ * MMF_ERR_PLAN if a program run refused its workspace (and nothing timed out), or
  * MMF_ERR_CUDA if the read itself failed. */
 mmf_status mmf_get_device_status(void);
 

@@ -80,4 +80,8 @@ WORKLOADS = {w.name: w for w in [
     HGRN_1P3B_PREFILL, HGRN_2P7B_DECODE_T8, HGRN_2P7B_PREFILL,
 ]}
 
-DEFAULT = HGRN_370M_T64.name
+# the largest configuration that fits one GPU: the benchmark's headline workload
+DEFAULT = HGRN_1P3B_PREFILL.name
+# the decode configurations the benchmark reports beside it (HBM-bound regime)
+DECODE_SUITE = ("hgrn1p3b_decode_t1", "hgrn1p3b_decode_t8", "hgrn1p3b_decode_t64",
+                "hgrn2p7b_decode_t8")

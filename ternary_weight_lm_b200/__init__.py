@@ -33,6 +33,7 @@ MMF_F16 = 1
 STATUS = {
     0: "MMF_OK", 1: "MMF_ERR_INVALID_ARG", 2: "MMF_ERR_UNSUPPORTED_SHAPE",
     3: "MMF_ERR_ALIGNMENT", 4: "MMF_ERR_CUDA", 5: "MMF_ERR_TIMEOUT", 6: "MMF_ERR_WORKSPACE",
+    7: "MMF_ERR_RESOURCES", 8: "MMF_ERR_PLAN",
 }
 
 

@@ -11,6 +11,11 @@ namespace mmf {
 enum InDType { kInF32 = 0, kInF16 = 1 };
 enum OutMode { kOutF32 = 0, kOutF16 = 1, kOutI32 = 2 };
 
+// Per-device host tables (status word address, one-time kernel attributes) have this many
+// slots; a call made with a current device of this index or above fails with a CUDA error
+// instead of sharing another device's slot.
+constexpr int kMaxDevices = 64;
+
 // Default limit for any one device-side wait before a kernel gives up (nanoseconds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

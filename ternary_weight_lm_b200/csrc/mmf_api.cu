@@ -9,6 +9,7 @@
 
 #include "../../include/mmf.h"
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 #define MMF_EXPORT extern "C" __attribute__((visibility("default")))
 
@@ -66,17 +67,17 @@ FwdWs fwd_ws(void* ws, int64_t T, int64_t K) {
 }
 
 unsigned* status_ptr() {
-  static unsigned* ptrs[64] = {nullptr};
+  static unsigned* ptrs[kMaxDevices] = {nullptr};
   static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
-  if (ptrs[dev & 63] == nullptr) {
+  if (ptrs[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    ptrs[dev & 63] = reinterpret_cast<unsigned*>(p);
+    ptrs[dev] = reinterpret_cast<unsigned*>(p);
   }
-  return ptrs[dev & 63];
+  return ptrs[dev];
 }
 
 mmf_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MMF_OK : MMF_ERR_CUDA; }
@@ -298,7 +299,9 @@ MMF_EXPORT mmf_status mmf_get_device_status(void) {
   if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return MMF_ERR_CUDA;
   const unsigned zero = 0;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return MMF_ERR_CUDA;
-  return (v & 1u) ? MMF_ERR_TIMEOUT : MMF_OK;
+  if (v & kStatusTimeout) return MMF_ERR_TIMEOUT;
+  if (v & kStatusBadPlan) return MMF_ERR_PLAN;
+  return MMF_OK;
 }
 
 MMF_EXPORT mmf_status mmf_debug_wait_timeout_probe(uint64_t limit_ns, void* stream) {
@@ -317,6 +320,8 @@ MMF_EXPORT const char* mmf_status_string(mmf_status s) {
     case MMF_ERR_CUDA: return "MMF_ERR_CUDA";
     case MMF_ERR_TIMEOUT: return "MMF_ERR_TIMEOUT";
     case MMF_ERR_WORKSPACE: return "MMF_ERR_WORKSPACE";
+    case MMF_ERR_RESOURCES: return "MMF_ERR_RESOURCES";
+    case MMF_ERR_PLAN: return "MMF_ERR_PLAN";
   }
   return "MMF_ERR_UNKNOWN";
 }

@@ -35,10 +35,10 @@ size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 // Device address of the scratch array for the current device, looked up once per device.
 unsigned char* noalloc_scratch_ptr() {
-  static unsigned char* ptrs[64] = {nullptr};
+  static unsigned char* ptrs[kMaxDevices] = {nullptr};
   static std::mutex mu;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lk(mu);
   if (ptrs[dev] == nullptr) {
     unsigned char* p = nullptr;

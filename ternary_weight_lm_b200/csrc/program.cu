@@ -61,6 +61,8 @@ constexpr int kMaxProj = 1024;
 constexpr int kMaxSplit = 16;
 constexpr int kMinSplitKb = 32;            // a split tile costs a few microseconds of reduction
 constexpr uint64_t kPDrainNs = 2000000000ull;
+constexpr uint32_t kPlanMagic = 0x4d4d4650u;   // "PFMM"
+
 static_assert(kPACol0 + kPSlots * 32 == 512, "TMEM columns");
 // Two partial accumulators per unit (even / odd sub-blocks) when they fit in the unit's 64
 // accumulator columns.
@@ -113,7 +115,9 @@ constexpr int kERecMax = 128;
 struct PHeader {
   int32_t n_proj, n_in, n_levels, n_ctas, n_units, T, BN, n_tiles;
   float eps;
-  int32_t pad[3];
+  uint32_t magic;       // kPlanMagic once a plan is written
+  uint32_t gen;         // init generation: every run passes the generation it was planned with
+  int32_t pad;
   int64_t off_in, off_proj, off_units, off_ctaoff, off_wt, off_tilectr, off_levelctr, off_part;
   int64_t off_erec;
   int32_t in_begin[kMaxLevels + 1];
@@ -474,7 +478,7 @@ __device__ __forceinline__ void load_acc_sum(uint32_t taddr, int mask, int32_t (
 
 template <int BN>
 __global__ void __launch_bounds__(kPThreads, 1)
-program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_ns) {
+program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, uint64_t limit_ns) {
   using C = PCfg<BN>;
   constexpr int S = C::kStages;
   // With BN <= 32 two MMA warps on different SM sub-partitions take alternate stages, each into
@@ -541,6 +545,19 @@ program_kernel(const uint8_t* __restrict__ ws, unsigned* status, uint64_t limit_
   pdl_wait();
   // the plan in the workspace is read only after the wait
   const PHeader& H = *reinterpret_cast<const PHeader*>(ws);
+  // A workspace that does not hold the plan this launch was made for (never planned, planned
+  // again for another program, or overwritten) is refused by every CTA alike: nothing is
+  // read or written beyond the header, and the status word records it.
+  if (H.magic != kPlanMagic || H.gen != gen || H.BN != BN || H.n_ctas != static_cast<int>(gridDim.x)) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(status, kStatusBadPlan);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+    return;
+  }
   const PIn* ins = reinterpret_cast<const PIn*>(ws + H.off_in);
   const PProj* projs = reinterpret_cast<const PProj*>(ws + H.off_proj);
   const PUnit* units = reinterpret_cast<const PUnit*>(ws + H.off_units);
@@ -1333,35 +1350,112 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
 struct RunInfo {
   int BN;
   int nct;
+  uint32_t gen;   // the plan's generation, also written into the workspace header
+  int mode;       // launch attributes (see launch_mode)
 };
 std::mutex g_runs_mu;
 std::unordered_map<const void*, RunInfo> g_runs;
+uint32_t g_next_gen = 1;
 
 template <int BN>
-cudaError_t launch_program(const void* ws, int nct, unsigned* status, cudaStream_t s) {
+cudaError_t set_program_attr() {
   using C = PCfg<BN>;
-  static std::once_flag once[64];
+  static std::once_flag once[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   cudaError_t ae = cudaSuccess;
-  std::call_once(once[dev & 63], [&] {
+  std::call_once(once[dev], [&] {
     ae = cudaFuncSetAttribute(program_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               C::kSmem);
   });
+  return ae;
+}
+
+// CTAs of program_kernel<BN> one device can hold at once (0 on failure).
+template <int BN>
+int resident_ctas() {
+  using C = PCfg<BN>;
+  if (set_program_attr<BN>() != cudaSuccess) return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, program_kernel<BN>, kPThreads,
+                                                    C::kSmem) != cudaSuccess)
+    return 0;
+  return per_sm * sm_count();
+}
+
+int resident_ctas_for(int BN) {
+  return BN == 16 ? resident_ctas<16>() : (BN == 32 ? resident_ctas<32>() : resident_ctas<64>());
+}
+
+__global__ void launch_mode_probe_kernel() {}
+
+// Launch attributes every program run uses on this device, found once (outside any stream
+// capture: mmf_program_init is never captured) by launching an empty kernel with them.  A
+// cooperative launch makes the driver place every CTA of the grid at once, which the grid
+// barriers need; programmatic serialisation lets the launch's set-up overlap the tail of the
+// previous kernel on the stream.  Bit 0: cooperative, bit 1: programmatic serialisation.
+int launch_mode(cudaStream_t s) {
+  static int modes[kMaxDevices];
+  static std::once_flag once[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::call_once(once[dev], [&] {
+    const int tries[3] = {3, 1, 2};
+    modes[dev] = 0;
+    for (int m : tries) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1);
+      cfg.blockDim = dim3(32);
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      int na = 0;
+      if (m & 1) {
+        attr[na].id = cudaLaunchAttributeCooperative;
+        attr[na++].val.cooperative = 1;
+      }
+      if (m & 2) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na++].val.programmaticStreamSerializationAllowed = 1;
+      }
+      cfg.attrs = attr;
+      cfg.numAttrs = na;
+      if (cudaLaunchKernelEx(&cfg, launch_mode_probe_kernel) == cudaSuccess) {
+        modes[dev] = m;
+        break;
+      }
+      (void)cudaGetLastError();   // a refused configuration is not sticky
+    }
+  });
+  return modes[dev];
+}
+
+template <int BN>
+cudaError_t launch_program(const void* ws, int nct, uint32_t gen, int mode, unsigned* status,
+                           cudaStream_t s) {
+  using C = PCfg<BN>;
+  cudaError_t ae = set_program_attr<BN>();
   if (ae != cudaSuccess) return ae;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(nct));
   cfg.blockDim = dim3(kPThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, program_kernel<BN>, reinterpret_cast<const uint8_t*>(ws), status,
-                            kWaitLimitNs);
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (mode & 1) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na++].val.cooperative = 1;
+  }
+  if (mode & 2) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na++].val.programmaticStreamSerializationAllowed = 1;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, program_kernel<BN>, reinterpret_cast<const uint8_t*>(ws), gen,
+                            status, kWaitLimitNs);
 }
 
 }  // namespace
@@ -1387,6 +1481,19 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   st = build_plan(p, n, T, eps, reinterpret_cast<uintptr_t>(ws), nct, P);
   if (st != MMF_OK) return st;
   if (ws_bytes < P.bytes) return MMF_ERR_WORKSPACE;
+  // Every CTA of a run waits for all the others at the level barriers: the device must be able
+  // to hold the whole grid at once.
+  if (resident_ctas_for(P.BN) < nct) return MMF_ERR_RESOURCES;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int mode = launch_mode(s);
+  uint32_t gen;
+  {
+    std::lock_guard<std::mutex> lk(g_runs_mu);
+    gen = g_next_gen++;
+    if (g_next_gen == 0) g_next_gen = 1;
+  }
+  P.h.magic = kPlanMagic;
+  P.h.gen = gen;
   // host image of the plan region, copied in one stream-ordered copy; counters zeroed
   const size_t plan_end = static_cast<size_t>(P.h.off_levelctr) + (2 * kMaxLevels + 2) * 4;
   std::vector<uint8_t> img(plan_end, 0);
@@ -1396,7 +1503,6 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   std::memcpy(img.data() + P.h.off_units, P.units.data(), P.units.size() * sizeof(PUnit));
   std::memcpy(img.data() + P.h.off_erec, P.erec.data(), P.erec.size() * sizeof(PERec));
   std::memcpy(img.data() + P.h.off_ctaoff, P.ctaoff.data(), P.ctaoff.size() * sizeof(int32_t));
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // pageable source: the copy has consumed the host buffer when cudaMemcpyAsync returns
   if (cudaMemcpyAsync(ws, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
     return MMF_ERR_CUDA;
@@ -1414,7 +1520,7 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
     return MMF_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lk(g_runs_mu);
-    g_runs[ws] = RunInfo{P.BN, nct};
+    g_runs[ws] = RunInfo{P.BN, nct, gen, mode};
   }
   return MMF_OK;
 }
@@ -1433,10 +1539,14 @@ MMF_EXPORT mmf_status mmf_program_run(void* ws, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (ri.BN == 16)
-    e = launch_program<16>(ws, ri.nct, status, s);
+    e = launch_program<16>(ws, ri.nct, ri.gen, ri.mode, status, s);
   else if (ri.BN == 32)
-    e = launch_program<32>(ws, ri.nct, status, s);
+    e = launch_program<32>(ws, ri.nct, ri.gen, ri.mode, status, s);
   else
-    e = launch_program<64>(ws, ri.nct, status, s);
+    e = launch_program<64>(ws, ri.nct, ri.gen, ri.mode, status, s);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return MMF_ERR_RESOURCES;
+  }
   return e == cudaSuccess ? MMF_OK : MMF_ERR_CUDA;
 }

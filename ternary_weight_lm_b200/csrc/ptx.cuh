@@ -9,6 +9,8 @@ namespace mmf {
 
 // Device status word bits (OR-ed into the word the caller passes to each kernel).
 constexpr unsigned kStatusTimeout = 1u;
+// A persistent launch found a workspace that does not hold the plan it was launched for.
+constexpr unsigned kStatusBadPlan = 2u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

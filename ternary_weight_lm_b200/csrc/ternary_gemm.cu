@@ -456,12 +456,13 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
 template <int BN, int TC = 512>
 cudaError_t launch_bn(const GemmCall& c, cudaStream_t s) {
   using Cf = Cfg<BN, TC>;
-  static std::once_flag attr_once[64];
+  static std::once_flag attr_once[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once[dev & 63], [&] {
+  std::call_once(attr_once[dev], [&] {
     attr_err = cudaFuncSetAttribute(ternary_gemm_kernel<BN, TC>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmem);
   });

@@ -108,3 +108,25 @@ def test_valid_call_without_gpu_reports_cuda_error():
     assert fwd() == CUDA
     with pytest.raises(mmf.MMFError):
         mmf._check("mmf_bitlinear_forward", fwd())
+
+
+def test_program_run_refuses_a_workspace_without_a_plan():
+    # A workspace that no successful mmf_program_init planned is refused on the host, before
+    # any launch (the run could not know the plan's token tile or grid).
+    L = mmf.lib()
+    assert L.mmf_program_run(A16, None) == INVALID
+    assert L.mmf_program_run(None, None) == INVALID
+
+
+def test_program_init_rejects_on_host():
+    L = mmf.lib()
+    p = mmf.Projection(A16, 1, None, A16, A16, 256, 256, 0, 0, A16, 1)
+    arr = (mmf.Projection * 1)(p)
+    assert L.mmf_program_init(arr, 1, 65, 1e-8, A16, 1 << 30, None) == SHAPE   # T > 64
+    assert L.mmf_program_init(arr, 1, 8, 0.0, A16, 1 << 30, None) == INVALID   # eps
+    assert L.mmf_program_init(arr, 0, 8, 1e-8, A16, 1 << 30, None) == INVALID  # no projection
+    assert L.mmf_program_init(arr, 1, 8, 1e-8, None, 1 << 30, None) == WS
+    assert L.mmf_program_init(arr, 1, 8, 1e-8, A16 + 16, 1 << 30, None) == ALIGN
+    bad = (mmf.Projection * 1)(mmf.Projection(A16, 1, None, A16, A16, 200, 256, 0, 0, A16, 1))
+    assert L.mmf_program_init(bad, 1, 8, 1e-8, A16, 1 << 30, None) == SHAPE      # K % 128
+    assert L.mmf_program_workspace_bytes(bad, 1, 8) == 0

@@ -130,6 +130,10 @@ def test_accumulate_i32_extremes():
     (64, 2816, 1024, np.float16, torch.float16),
     (77, 640, 384, np.float16, torch.float32),
     (300, 1024, 256, np.float16, torch.float16),
+    # the 2.7B-shaped down_proj (K = 7040, a partial last 512-wide k stage) at decode and
+    # above the 256-token tile
+    (8, 7040, 2560, np.float16, torch.float16),
+    (300, 7040, 2560, np.float16, torch.float16),
 ])
 def test_forward_parity(T, K, N, dt, odt):
     x = synth.activations(T + N, f"fw{T}", T, K, dtype=dt)
@@ -188,6 +192,12 @@ def test_block_projections_370m_t64():
             h_gpu, h_ref = y, y_ref
 
 
+def _sampled_rows(T, n, seed):
+    rows = np.random.default_rng(seed).choice(T, n, replace=False)
+    rows[0], rows[-1] = 0, T - 1
+    return rows
+
+
 def test_prefill_sampled_rows_1p3b_gate():
     """The 1.3B prefill gate_proj at full size (32768 tokens, 1 % outliers x20): every
     activation code, and every output of 24 sampled token rows, against the oracle."""
@@ -200,10 +210,32 @@ def test_prefill_sampled_rows_1p3b_gate():
     q_ref, gamma_ref, _ = oracle.rmsnorm_actquant(x)
     assert_codes_close(A, q_ref)
     h = gpu_forward(x, Wp, beta, glu=True)
-    rows = np.random.default_rng(1).choice(T, 24, replace=False)
-    rows[0], rows[-1] = 0, T - 1
+    rows = _sampled_rows(T, 24, 1)
     h_ref = oracle_forward_from_parts(x[rows], Wp, beta, K, glu=True)
     assert_out_close(h[rows], h_ref)
+
+
+def test_prefill_sampled_rows_2p7b_gate_and_down():
+    """The 2.7B prefill shapes at full size: gate_proj 2560 -> 14080 with the GLU at 8192
+    tokens, then down_proj 7040 -> 2560 fed by its fp16 GLU output.  Every activation code of
+    both inputs, and 16 sampled token rows of both outputs, against the oracle."""
+    T, H, I = 8192, 2560, 7040
+    x = synth.activations(0, "prefill27", T, H)
+    Wg = synth.weights(0, "prefill27_gate", 2 * I, H)
+    Wd = synth.weights(0, "prefill27_down", H, I)
+    Wpg, bg = gpu_quantize_weights(Wg)
+    Wpd, bd = gpu_quantize_weights(Wd)
+    assert bg == oracle.absmean_beta(Wg) and bd == oracle.absmean_beta(Wd)
+    rows = _sampled_rows(T, 16, 2)
+    A, _, _ = gpu_act_quant(x)
+    assert_codes_close(A, oracle.rmsnorm_actquant(x)[0])
+    h = gpu_forward(x, Wpg, bg, glu=True)
+    assert_out_close(h[rows], oracle_forward_from_parts(x[rows], Wpg, bg, H, glu=True))
+    h16 = h.astype(np.float16)                  # down_proj reads the fp16 GLU output
+    A, _, _ = gpu_act_quant(h16)
+    assert_codes_close(A, oracle.rmsnorm_actquant(h16)[0])
+    y = gpu_forward(h16, Wpd, bd)
+    assert_out_close(y[rows], oracle_forward_from_parts(h16[rows], Wpd, bd, I))
 
 
 # ---------------------------------------------------------------------------- status

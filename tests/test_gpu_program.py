@@ -79,22 +79,50 @@ def test_program_370m_block_matches_single_calls_and_oracle(T):
         assert_out_close(p["y"].double().cpu().numpy(), y_ref)
 
 
+def _check_against_oracle(projs, host, norm=False):
+    """Every projection of a run program against the oracle's projection, each fed the
+    program's own fp16/fp32 input (for a chained input, the program's earlier output)."""
+    for i, ((spec, Wp, beta), p) in enumerate(zip(host, projs)):
+        g = p["norm_w"].cpu().numpy() if norm and p["norm_w"] is not None else None
+        y_ref = oracle_forward_from_parts(p["x"].cpu().numpy(), Wp.cpu().numpy(),
+                                          float(beta.item()), spec.K, g=g, glu=spec.glu)
+        try:
+            assert_out_close(p["y"].double().cpu().numpy(), y_ref)
+        except AssertionError as e:
+            raise AssertionError(f"projection {i} ({spec.name}): {e}") from None
+
+
 def test_program_two_chained_1p3b_layers():
+    """Two 1.3B-shaped layers chained (layer 2's i/f/g read layer 1's down_proj output): four
+    dependency levels.  Each projection matches the single-projection entry point bit for bit
+    and the oracle within the output tolerance, both fed the program's own inputs."""
     T = 8
     projs, host = _block(2048, 5632, T, seed=3, layers=2, chain=True)
     prog = mmf.Program(projs, T)
     prog.run()
     torch.cuda.synchronize()
     assert mmf.mmf_get_device_status() == 0
-    ref = _reference_outputs([dict(p, y=torch.empty_like(p["y"])) for p in projs])
-    # chained inputs: the reference reads the program's own intermediate outputs, so compare
-    # level by level using the program's inputs
     for i, p in enumerate(projs):
         f = mmf.bitlinear_glu_forward if p["glu"] else mmf.bitlinear_forward
         y1 = f(p["x"], p["Wp"], p["beta"], out_dtype=p["y"].dtype)
         torch.cuda.synchronize()
         np.testing.assert_array_equal(p["y"].cpu().numpy(), y1.cpu().numpy(), err_msg=f"proj {i}")
-    del ref
+    _check_against_oracle(projs, host)
+
+
+@pytest.mark.parametrize("T", [1, 8, 16])
+def test_program_2p7b_block_against_oracle(T):
+    """A 2.7B-shaped block (hidden 2560, GLU half 7040): down_proj's K = 7040 ends in a partial
+    512-wide stage.  Run twice; every projection against the oracle."""
+    projs, host = _block(2560, 7040, T, seed=27 + T)
+    prog = mmf.Program(projs, T)
+    for rep in range(2):
+        for p in projs:
+            p["y"].fill_(float("nan"))
+        prog.run()
+        torch.cuda.synchronize()
+        assert mmf.mmf_get_device_status() == 0
+        _check_against_oracle(projs, host)
 
 
 def test_program_fp32_inputs_with_norm_weights():
@@ -145,3 +173,24 @@ def test_program_short_rows_and_partial_stages(T):
         y_ref = oracle_forward_from_parts(p["x"].cpu().numpy(), Wp.cpu().numpy(),
                                           float(beta.item()), K, glu=glu)
         assert_out_close(p["y"].double().cpu().numpy(), y_ref)
+
+
+def test_program_refuses_a_workspace_whose_plan_was_overwritten():
+    """A run whose workspace no longer holds its plan (here the header is zeroed after the
+    init) must not touch anything: every CTA returns at once and the status word reports
+    MMF_ERR_PLAN.  A fresh init makes the same workspace usable again."""
+    T = 4
+    projs, host = _block(1024, 2816, T, seed=71)
+    prog = mmf.Program(projs, T)
+    for p in projs:
+        p["y"].fill_(float("nan"))
+    prog.ws[:256].zero_()
+    prog.run()
+    torch.cuda.synchronize()
+    assert mmf.mmf_get_device_status() == 8          # MMF_ERR_PLAN
+    assert all(torch.isnan(p["y"].float()).all() for p in projs)
+    mmf.mmf_program_init(projs, T, 1e-8, prog.ws)
+    prog.run()
+    torch.cuda.synchronize()
+    assert mmf.mmf_get_device_status() == 0
+    _check_against_oracle(projs, host)

@@ -41,12 +41,18 @@ def test_dense_matmul_worked_example():
     np.testing.assert_array_equal(C, m["C"])
 
 
-def test_dense_matmul_transposes_fail():
-    # The example is not symmetric: A^T B^T gives a different 3x3 matrix, so an operand
-    # transposed by mistake cannot pass the pin above.
+def test_dense_matmul_transposes_and_operand_order():
+    # (A B)^T = B^T A^T: the page's product, transposed, must come out of the transposed and
+    # swapped operands.  The example is rectangular and not symmetric, so an oracle that read
+    # either operand with its indices swapped, or walked the inner index of one operand
+    # backwards, cannot meet both this and the pin above.
     m = _golden_matmul()
-    C = oracle.dense_matmul_i64(m["B"], m["A"])
-    assert C.shape == (3, 3)
+    np.testing.assert_array_equal(oracle.dense_matmul_i64(m["B"].T, m["A"].T), m["C"].T)
+    assert not np.array_equal(oracle.dense_matmul_i64(m["A"], m["B"][::-1]), m["C"])
+    assert not np.array_equal(oracle.dense_matmul_i64(m["A"][:, ::-1], m["B"]), m["C"])
+    # the swapped product B A is the 3x3 matrix worked out by hand from the page's entries
+    np.testing.assert_array_equal(oracle.dense_matmul_i64(m["B"], m["A"]),
+                                  [[39, 54, 69], [49, 68, 87], [59, 82, 105]])
 
 
 # ----------------------------------------------------------------------------------------------

@@ -1,6 +1,7 @@
 """The allocation-free forward (mmf_bitlinear_forward_noalloc), for callers that cannot call
-cudaMalloc: its output must match the workspace-taking mmf_bitlinear_forward on the same
-inputs, on two calls in a row (the second call reuses the shared scratch left by the first).
+cudaMalloc: its output must equal, bit for bit, that of the workspace-taking
+mmf_bitlinear_forward on the same inputs, on two calls in a row (the second call reuses the
+shared scratch left by the first).
 Collected last on purpose, so a run that stops at the first failure has run everything else.
 """
 import ctypes
@@ -11,31 +12,45 @@ import torch
 
 import synth
 import ternary_weight_lm_b200 as mmf
-from gpu_helpers import DEV, assert_out_close, to_dev
+from gpu_helpers import DEV, assert_out_close, oracle_forward_from_parts, to_dev
 
 SCRATCH_BYTES = 4 << 20
 
 
-def _noalloc(x, Wp, beta, N, y):
+def _noalloc(x, Wp, beta, N, y, norm_w=None):
     T, K = x.shape
+    dt = {torch.float16: mmf.MMF_F16, torch.float32: mmf.MMF_F32}
     return mmf.lib().mmf_bitlinear_forward_noalloc(
-        x.data_ptr(), mmf.MMF_F16, T, K, None, ctypes.c_float(1e-8), Wp.data_ptr(),
-        beta.data_ptr(), N, y.data_ptr(), mmf.MMF_F16, torch.cuda.current_stream().cuda_stream)
+        x.data_ptr(), dt[x.dtype], T, K, None if norm_w is None else norm_w.data_ptr(),
+        ctypes.c_float(1e-8), Wp.data_ptr(), beta.data_ptr(), N, y.data_ptr(), dt[y.dtype],
+        torch.cuda.current_stream().cuda_stream)
 
 
 @pytest.mark.gpu
 def test_noalloc_matches_forward_on_two_calls():
-    cases = [(64, 1024, 1024, "first"), (17, 2816, 1024, "second")]
-    for T, K, N, label in cases:
-        x = to_dev(synth.activations(11, f"noalloc/{label}", T, K))
+    # The allocation-free call runs the same two kernels on the same inputs as
+    # mmf_bitlinear_forward, only with its scratch elsewhere, so the outputs must agree bit for
+    # bit.  Two calls in a row: the second one finds the first one's codes in the shared array.
+    # The second call also covers fp32 in, fp32 out and a non-trivial norm weight.
+    cases = [(64, 1024, 1024, "first", torch.float16, False),
+             (17, 2816, 1024, "second", torch.float32, True)]
+    for T, K, N, label, dt, with_g in cases:
+        xnp = synth.activations(11, f"noalloc/{label}", T, K,
+                                dtype=np.float32 if dt == torch.float32 else np.float16)
+        x = to_dev(xnp)
         W = to_dev(synth.weights(11, f"noalloc/{label}", N, K))
+        g = to_dev(synth.norm_weight(11, f"noalloc/{label}", K, ones=False)) if with_g else None
         Wp, beta = mmf.quantize_weights(W)
-        y_ref = mmf.bitlinear_forward(x, Wp, beta)            # the existing entry point
-        y = torch.full((T, N), float("nan"), dtype=torch.float16, device=DEV)
-        assert _noalloc(x, Wp, beta, N, y) == 0
+        y_ref = mmf.bitlinear_forward(x, Wp, beta, norm_w=g, out_dtype=dt)   # existing entry
+        y = torch.full((T, N), float("nan"), dtype=dt, device=DEV)
+        assert _noalloc(x, Wp, beta, N, y, norm_w=g) == 0
         torch.cuda.synchronize()
         assert torch.isfinite(y).all()
-        assert_out_close(y.double().cpu().numpy(), y_ref.double().cpu().numpy())
+        assert torch.equal(y, y_ref), f"{label}: differs from mmf_bitlinear_forward"
+        # and within the parity tolerance of the oracle
+        y_orc = oracle_forward_from_parts(xnp, Wp.cpu().numpy(), float(beta.item()), K,
+                                          g=None if g is None else g.cpu().numpy())
+        assert_out_close(y.double().cpu().numpy(), y_orc)
     assert mmf.mmf_get_device_status() == 0
 
 
