@@ -95,8 +95,9 @@ mmf_status mmf_ternary_encode(const void* W, mmf_dtype wdt, int64_t N, int64_t K
 
 /* ---- forward ([P1], [P3]; [P4] figure items 4 and 5) ------------------------------------ */
 
-/* Workspace bytes one forward call with T tokens, K inputs and N outputs needs: the int8
- * activation codes [T x K], gamma [T] and the code row sums [T], each 256-byte aligned. */
+/* Workspace bytes one forward call with T tokens, K inputs and N weight rows needs: the int8
+ * activation codes [T x K], gamma [T] and the code row sums [T], each 256-byte aligned, and
+ * for T > 128 (the prefill contraction) the weight codes expanded to int8 [N x K]. */
 size_t mmf_forward_workspace_bytes(int64_t T, int64_t K, int64_t N);
 
 /* y [T x N] = FusedBitLinear(x [T x K]).  xdt: f32 or f16.  norm_w: K floats or NULL
@@ -124,14 +125,22 @@ mmf_status mmf_quantize_activations(const void* x, mmf_dtype xdt, int64_t T, int
                                     const float* norm_w, float eps, int8_t* A, float* gamma,
                                     int32_t* rowsum, void* stream);
 
+/* Workspace bytes mmf_bitlinear_forward_quantized needs for the prefill contraction: the weight
+ * codes expanded to int8 [N x K] when T > 128, else 0. */
+size_t mmf_quantized_workspace_bytes(int64_t T, int64_t K, int64_t N);
+
 /* Second half of the forward: contraction + dequantisation (+ SiLU-GLU when glu != 0, then
  * N is 2I and y is T x I) from activation codes already produced by mmf_quantize_activations
- * (A [T x K], gamma [T], rowsum [T]).  One launch.  Lets callers reuse one quantised input
- * for several projections whose norm weights are equal. */
+ * (A [T x K], gamma [T], rowsum [T]).  Lets callers reuse one quantised input for several
+ * projections whose norm weights are equal.  ws: NULL with ws_bytes 0 (the contraction that
+ * needs no workspace), or mmf_quantized_workspace_bytes(T, K, N) bytes, 256-byte aligned;
+ * for T > 128 and N % 256 == 0 the latter selects the faster prefill contraction, which first
+ * expands the packed codes into ws.  Same results either way. */
 mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const float* gamma,
                                            const int32_t* rowsum, int64_t T, int64_t K,
                                            const uint8_t* Wp, const float* beta, int64_t N,
-                                           int glu, void* y, mmf_dtype ydt, void* stream);
+                                           int glu, void* y, mmf_dtype ydt, void* ws,
+                                           size_t ws_bytes, void* stream);
 
 /* acc [T x N] int32 = ternary accumulation of given codes A [T x K] against Wp.  Exact.
  * ws must hold mmf_forward_workspace_bytes(T, K, N). */

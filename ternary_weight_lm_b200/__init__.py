@@ -17,7 +17,8 @@ __all__ = [
     "MMFError", "lib", "lib_path",
     "mmf_quantize_weights_workspace_bytes", "mmf_quantize_weights", "mmf_ternary_encode",
     "mmf_forward_workspace_bytes", "mmf_bitlinear_forward", "mmf_bitlinear_glu_forward",
-    "mmf_quantize_activations", "mmf_bitlinear_forward_quantized",
+    "mmf_quantize_activations", "mmf_quantized_workspace_bytes",
+    "mmf_bitlinear_forward_quantized",
     "mmf_ternary_accumulate_i32", "mmf_bitlinear_forward_noalloc", "mmf_get_device_status",
     "mmf_debug_wait_timeout_probe", "mmf_status_string", "mmf_version",
     "mmf_program_workspace_bytes", "mmf_program_init", "mmf_program_run", "Projection",
@@ -71,7 +72,9 @@ def lib():
             "mmf_bitlinear_forward": ([P, I, I64, I64, P, F, P, P, I64, P, I, P, SZ, P], I),
             "mmf_bitlinear_glu_forward": ([P, I, I64, I64, P, F, P, P, I64, P, I, P, SZ, P], I),
             "mmf_quantize_activations": ([P, I, I64, I64, P, F, P, P, P, P], I),
-            "mmf_bitlinear_forward_quantized": ([P, P, P, I64, I64, P, P, I64, I, P, I, P], I),
+            "mmf_quantized_workspace_bytes": ([I64, I64, I64], SZ),
+            "mmf_bitlinear_forward_quantized": ([P, P, P, I64, I64, P, P, I64, I, P, I, P, SZ, P],
+                                                I),
             "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
             "mmf_bitlinear_forward_noalloc": ([P, I, I64, I64, P, F, P, P, I64, P, I, P], I),
             "mmf_program_workspace_bytes": ([P, I, I64], SZ),
@@ -168,11 +171,18 @@ def mmf_quantize_activations(x, norm_w, eps, A, gamma, rowsum=None, stream=None)
         _stream(stream)))
 
 
-def mmf_bitlinear_forward_quantized(A, gamma, rowsum, Wp, beta, N, glu, y, stream=None):
+def mmf_quantized_workspace_bytes(T, K, N):
+    return lib().mmf_quantized_workspace_bytes(T, K, N)
+
+
+def mmf_bitlinear_forward_quantized(A, gamma, rowsum, Wp, beta, N, glu, y, ws=None,
+                                    stream=None):
+    """ws: None (the contraction that needs no workspace) or a tensor of at least
+    mmf_quantized_workspace_bytes(T, K, N) bytes."""
     T, K = A.shape
     _check("mmf_bitlinear_forward_quantized", lib().mmf_bitlinear_forward_quantized(
         _ptr(A), _ptr(gamma), _ptr(rowsum), T, K, _ptr(Wp), _ptr(beta), N, 1 if glu else 0,
-        _ptr(y), _dt(y), _stream(stream)))
+        _ptr(y), _dt(y), _ptr(ws), 0 if ws is None else _nbytes(ws), _stream(stream)))
 
 
 def mmf_ternary_accumulate_i32(A, Wp, N, acc, ws, stream=None):

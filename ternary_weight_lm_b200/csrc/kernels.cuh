@@ -48,8 +48,15 @@ struct GemmCall {
   int out_mode;           // OutMode
   unsigned* status;
   uint64_t wait_limit_ns;
+  int8_t* w8 = nullptr;   // scratch of prefill_w8_bytes(rows, K) for the int8 weight codes, or
+                          // nullptr (then no kernel needs it)
 };
 cudaError_t launch_ternary_gemm(const GemmCall& c, cudaStream_t s);
+
+// The prefill contraction as a CTA-pair int8 GEMM: needs T > 128, rows % 256 == 0 and w8.
+size_t prefill_w8_bytes(int64_t N, int64_t K);
+bool prefill_ss_supported(const GemmCall& c);
+cudaError_t launch_prefill_ss(const GemmCall& c, int8_t* w8, cudaStream_t s);
 
 // Device address of the library's status word on the current device (nullptr on failure).
 unsigned* device_status_word();
@@ -57,7 +64,11 @@ unsigned* device_status_word();
 // One block, one wait that nothing satisfies: must give up after limit_ns.
 cudaError_t launch_wait_probe(uint64_t limit_ns, unsigned* status, cudaStream_t s);
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).  Sizes
+// and box extents in elements of `dt`, the row stride in bytes.
+bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swz);
 bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                      CUtensorMapSwizzle swz);

@@ -49,13 +49,20 @@ struct FwdWs {
   int8_t* A;
   float* gamma;
   int32_t* rowsum;
+  int8_t* w8;      // int8 weight codes for the prefill contraction (nullptr when not needed)
 };
 
-size_t fwd_ws_bytes(int64_t T, int64_t K) {
-  return up256(static_cast<size_t>(T) * static_cast<size_t>(K)) + 2 * up256(static_cast<size_t>(T) * 4);
+// int8 weight codes: needed by the prefill contraction (more than 128 tokens)
+size_t w8_ws_bytes(int64_t T, int64_t K, int64_t N) {
+  return T > 128 ? up256(prefill_w8_bytes(N, K)) : 0;
 }
 
-FwdWs fwd_ws(void* ws, int64_t T, int64_t K) {
+size_t fwd_ws_bytes(int64_t T, int64_t K, int64_t N) {
+  return up256(static_cast<size_t>(T) * static_cast<size_t>(K)) +
+         2 * up256(static_cast<size_t>(T) * 4) + w8_ws_bytes(T, K, N);
+}
+
+FwdWs fwd_ws(void* ws, int64_t T, int64_t K, int64_t N) {
   uint8_t* b = reinterpret_cast<uint8_t*>(ws);
   FwdWs w;
   w.A = reinterpret_cast<int8_t*>(b);
@@ -63,6 +70,8 @@ FwdWs fwd_ws(void* ws, int64_t T, int64_t K) {
   w.gamma = reinterpret_cast<float*>(b);
   b += up256(static_cast<size_t>(T) * 4);
   w.rowsum = reinterpret_cast<int32_t*>(b);
+  b += up256(static_cast<size_t>(T) * 4);
+  w.w8 = w8_ws_bytes(T, K, N) ? reinterpret_cast<int8_t*>(b) : nullptr;
   return w;
 }
 
@@ -108,13 +117,13 @@ mmf_status fwd_common(const void* x, int xdt, int64_t T, int64_t K, const float*
   if (!aligned(x, 16) || !aligned(Wp, 16) || !aligned(y, 16) || !aligned(beta, 4) ||
       (norm_w && !aligned(norm_w, 16)))
     return MMF_ERR_ALIGNMENT;
-  if (!ws || ws_bytes < fwd_ws_bytes(T, K)) return MMF_ERR_WORKSPACE;
+  if (!ws || ws_bytes < fwd_ws_bytes(T, K, rows)) return MMF_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return MMF_ERR_ALIGNMENT;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   unsigned* status = status_ptr();
   if (!status) return MMF_ERR_CUDA;
-  FwdWs w = fwd_ws(ws, T, K);
+  FwdWs w = fwd_ws(ws, T, K, rows);
   cudaError_t e = launch_act_quant(x, xdt == MMF_F16 ? kInF16 : kInF32, T, static_cast<int>(K),
                                    norm_w, eps, w.A, w.gamma, w.rowsum, s);
   if (e != cudaSuccess) return MMF_ERR_CUDA;
@@ -132,6 +141,7 @@ mmf_status fwd_common(const void* x, int xdt, int64_t T, int64_t K, const float*
   c.out_mode = ydt == MMF_F16 ? kOutF16 : kOutF32;
   c.status = status;
   c.wait_limit_ns = kWaitLimitNs;
+  c.w8 = w.w8;
   return from_cuda(launch_ternary_gemm(c, s));
 }
 
@@ -139,19 +149,26 @@ mmf_status fwd_common(const void* x, int xdt, int64_t T, int64_t K, const float*
 
 unsigned* device_status_word() { return status_ptr(); }
 
-bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                     CUtensorMapSwizzle swz) {
+bool make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                  uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                     CUtensorMapSwizzle swz) {
+  return make_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, outer, row_bytes, box_inner,
+                      box_outer, swz);
 }
 
 }  // namespace mmf
@@ -193,9 +210,13 @@ MMF_EXPORT mmf_status mmf_ternary_encode(const void* W, mmf_dtype wdt, int64_t N
 }
 
 MMF_EXPORT size_t mmf_forward_workspace_bytes(int64_t T, int64_t K, int64_t N) {
-  (void)N;
-  if (T < 1 || K < 1) return 0;
-  return fwd_ws_bytes(T, K);
+  if (T < 1 || K < 1 || N < 1) return 0;
+  return fwd_ws_bytes(T, K, N);
+}
+
+MMF_EXPORT size_t mmf_quantized_workspace_bytes(int64_t T, int64_t K, int64_t N) {
+  if (T < 1 || K < 1 || N < 1) return 0;
+  return w8_ws_bytes(T, K, N);
 }
 
 MMF_EXPORT mmf_status mmf_bitlinear_forward(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
@@ -233,7 +254,7 @@ MMF_EXPORT mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const flo
                                                       const int32_t* rowsum, int64_t T, int64_t K,
                                                       const uint8_t* Wp, const float* beta,
                                                       int64_t N, int glu, void* y, mmf_dtype ydt,
-                                                      void* stream) {
+                                                      void* ws, size_t ws_bytes, void* stream) {
   if (!A || !gamma || !rowsum || !Wp || !beta || !y) return MMF_ERR_INVALID_ARG;
   if (check_dtype(ydt) != MMF_OK || (glu != 0 && glu != 1)) return MMF_ERR_INVALID_ARG;
   mmf_status st;
@@ -242,6 +263,10 @@ MMF_EXPORT mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const flo
   if (!aligned(A, 16) || !aligned(Wp, 16) || !aligned(y, 16) || !aligned(gamma, 4) ||
       !aligned(rowsum, 4) || !aligned(beta, 4))
     return MMF_ERR_ALIGNMENT;
+  // no workspace: the contraction that needs none; otherwise at least the queried size
+  if (ws != nullptr && ws_bytes < w8_ws_bytes(T, K, N)) return MMF_ERR_WORKSPACE;
+  if (ws == nullptr && ws_bytes != 0) return MMF_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned(ws, 256)) return MMF_ERR_ALIGNMENT;
   unsigned* status = status_ptr();
   if (!status) return MMF_ERR_CUDA;
   GemmCall c;
@@ -258,6 +283,7 @@ MMF_EXPORT mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const flo
   c.out_mode = ydt == MMF_F16 ? kOutF16 : kOutF32;
   c.status = status;
   c.wait_limit_ns = kWaitLimitNs;
+  c.w8 = (ws != nullptr && w8_ws_bytes(T, K, N) > 0) ? reinterpret_cast<int8_t*>(ws) : nullptr;
   return from_cuda(launch_ternary_gemm(c, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -269,12 +295,12 @@ MMF_EXPORT mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int
   if ((st = check_t(T)) != MMF_OK || (st = check_k(K)) != MMF_OK || (st = check_n(N)) != MMF_OK)
     return st;
   if (!aligned(A, 16) || !aligned(Wp, 16) || !aligned(acc, 16)) return MMF_ERR_ALIGNMENT;
-  if (!ws || ws_bytes < fwd_ws_bytes(T, K)) return MMF_ERR_WORKSPACE;
+  if (!ws || ws_bytes < fwd_ws_bytes(T, K, N)) return MMF_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return MMF_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   unsigned* status = status_ptr();
   if (!status) return MMF_ERR_CUDA;
-  FwdWs w = fwd_ws(ws, T, K);
+  FwdWs w = fwd_ws(ws, T, K, N);
   cudaError_t e = launch_rowsum(A, T, static_cast<int>(K), w.rowsum, s);
   if (e != cudaSuccess) return MMF_ERR_CUDA;
   GemmCall c;
@@ -291,6 +317,7 @@ MMF_EXPORT mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int
   c.out_mode = kOutI32;
   c.status = status;
   c.wait_limit_ns = kWaitLimitNs;
+  c.w8 = w.w8;
   return from_cuda(launch_ternary_gemm(c, s));
 }
 

@@ -42,28 +42,31 @@ constexpr int64_t kSplitTargetCtas = 148;       // SMs of a B200
 
 // TC: TMEM columns a CTA allocates.  512: one CTA owns the SM.  256: two CTAs share an SM
 // (half the shared memory each), so one CTA's epilogue overlaps the other's main loop.
+// The shared-memory ring (activation tile + packed weights per k-block) and the TMEM ring of
+// unpacked weight slots are separate: a stage is held from its copy's issue until its MMAs
+// complete, a slot only from its unpack until then.  The copies of a stage are L2 hits with
+// microseconds of latency under the prefill load, so the shared-memory ring is made as deep
+// as shared memory allows, whatever the number of TMEM slots.
 template <int BN, int TC = 512>
 struct Cfg {
   static constexpr int kActStage = BN * kKB;               // int8 activation tile
   static constexpr int kStage = kActStage + kWStageBytes;
-  // One ring: stage s of shared memory and slot s of TMEM (the unpacked weights of that
-  // stage) are filled and freed together, so every role waits on one barrier per k-block.
   static constexpr int kTmemCols = TC;
   static constexpr int kACol0 = ((BN + 31) / 32) * 32;     // first TMEM column of A slots
   static constexpr int kSlotsMax = (kTmemCols - kACol0) / 32;
+  static constexpr int kSlots = kSlotsMax > 16 ? 16 : kSlotsMax;
   static constexpr int kSmemBudget = TC == 512 ? 214 * 1024 : 108 * 1024;
   static constexpr int kStagesSmem = kSmemBudget / kStage;
-  static constexpr int kS0 = kStagesSmem < kSlotsMax ? kStagesSmem : kSlotsMax;
-  static constexpr int kStages = kS0 > 16 ? 16 : kS0;
+  static constexpr int kStages = kStagesSmem > 16 ? 16 : kStagesSmem;
   static constexpr int kChunk = BN < 32 ? BN : 32;         // epilogue token columns per pass
-  static constexpr int kBarBytes = 8 * (3 * kStages + 1);
+  static constexpr int kBarBytes = 8 * (2 * kStages + 2 * kSlots + 1);
   static constexpr int kTokBytes = 8 * BN;                 // per-token scale and code sum
   static constexpr int kSmemUsed = 1024 + kStages * kStage + kBarBytes + kTokBytes;
   // TC == 512: at least ~116 KB, so only one CTA lives on an SM (its TMEM allocation never
   // waits).  TC == 256: at most ~112 KB, so exactly two fit, and their TMEM halves fit too.
   static constexpr int kSmem =
       TC == 512 ? (kSmemUsed < 118 * 1024 ? 118 * 1024 : kSmemUsed) : kSmemUsed;
-  static_assert(kStages >= 4, "pipeline needs four stages");
+  static_assert(kStages >= 4 && kSlots >= 4, "pipeline needs four stages");
   static_assert(kSmem <= 227 * 1024, "shared memory per block");
   static_assert(TC == 512 || kSmem <= 112 * 1024, "two CTAs per SM");
   static_assert(kChunk * 128 * 4 <= kStages * kActStage, "epilogue staging must fit");
@@ -178,19 +181,24 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     r1 = r0 + 64;
   }
 
-  // full(s): the stage's TMA bytes landed.  afull(s): the four unpack warps wrote TMEM slot s
-  // (they did so after seeing full(s), so afull(s) also implies the activation tile is in).
-  // empty(s): the MMAs of the stage completed and the unpack warps read its packed weights.
+  // full(s): stage s's TMA bytes landed.  empty(s): the MMAs that read stage s's activation
+  // tile completed and the unpack warps read its packed weights.  afull(a): the four unpack
+  // warps wrote TMEM slot a (after seeing full of the same k-block, so it also implies that
+  // k-block's activation tile is in).  afree(a): the MMAs that read slot a completed.
   auto full = [&](int s) { return smem_u32(bars + s); };
-  auto afull = [&](int s) { return smem_u32(bars + C::kStages + s); };
-  auto empty = [&](int s) { return smem_u32(bars + 2 * C::kStages + s); };
-  const uint32_t accfull = smem_u32(bars + 3 * C::kStages);
+  auto empty = [&](int s) { return smem_u32(bars + C::kStages + s); };
+  auto afull = [&](int a) { return smem_u32(bars + 2 * C::kStages + a); };
+  auto afree = [&](int a) { return smem_u32(bars + 2 * C::kStages + C::kSlots + a); };
+  const uint32_t accfull = smem_u32(bars + 2 * C::kStages + 2 * C::kSlots);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(afull(s), 4);       // the four unpack warps
       mbar_init(empty(s), 1 + 4);   // the MMA commit + the four unpack warps
+    }
+    for (int a = 0; a < C::kSlots; ++a) {
+      mbar_init(afull(a), 4);       // the four unpack warps
+      mbar_init(afree(a), 1);       // the MMA commit
     }
     mbar_init(accfull, 1);
     s_abort = 0;
@@ -252,25 +260,22 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
     // lane issues each MMA and commit.
     constexpr uint32_t idesc = idesc_i8_u8s8(128, BN);
     const uint64_t bdesc0 = smem_desc_kmajor_sw128(smem_u32(s_act));
-    int s = 0;
-    uint32_t ph = 0;
     for (int kb = 0; kb < nkb; ++kb) {
-      const bool w = mbar_wait_bounded(afull(s), ph, p.wait_limit_ns, abort_flag, p.status);
+      const int s = kb % C::kStages, a = kb % C::kSlots;
+      const bool w = mbar_wait_bounded(afull(a), (kb / C::kSlots) & 1, p.wait_limit_ns,
+                                       abort_flag, p.status);
       if (!__all_sync(0xFFFFFFFFu, w)) break;
       tc_fence_after();
       // descriptor start address is in 16-byte units: a stage is kActStage bytes, a 32-deep
       // k step is 32 bytes within the 128-byte swizzled rows
       const uint64_t bd = bdesc0 + static_cast<uint64_t>((s * C::kActStage) >> 4);
-      const uint32_t ad = tmem + C::kACol0 + s * 32;
+      const uint32_t ad = tmem + C::kACol0 + a * 32;
       tc_mma_i8_ts_warp(tmem, ad, bd, idesc, kb > 0 ? 1u : 0u);   // kb counts this CTA's range
       tc_mma_i8_ts_warp(tmem, ad + 8, bd + 2, idesc, 1u);
       tc_mma_i8_ts_warp(tmem, ad + 16, bd + 4, idesc, 1u);
       tc_mma_i8_ts_warp(tmem, ad + 24, bd + 6, idesc, 1u);
       tc_commit_warp(empty(s));
-      if (++s == C::kStages) {
-        s = 0;
-        ph ^= 1u;
-      }
+      tc_commit_warp(afree(a));
     }
     // Signals the epilogue; in the abort path it also tells this warp when the MMAs it issued
     // have finished, so TMEM is not freed under them.
@@ -301,12 +306,10 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       }
     }
     bool ok = true;
-    int s = 0;
-    uint32_t ph = 0;
     for (int kb = 0; kb < nkb; ++kb) {
-      // full(s) of this use implies the previous use of stage s was released (the producer
-      // waited for it before reloading), so TMEM slot s is free as well.
-      const bool w = mbar_wait_bounded(full(s), ph, p.wait_limit_ns, abort_flag, p.status);
+      const int s = kb % C::kStages, a = kb % C::kSlots;
+      bool w = mbar_wait_bounded(full(s), (kb / C::kStages) & 1, p.wait_limit_ns, abort_flag,
+                                 p.status);
       if (!__all_sync(0xFFFFFFFFu, w)) {
         ok = false;
         break;
@@ -318,6 +321,15 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       const uint4 hi = *reinterpret_cast<const uint4*>(wrow + 16 * (sw ^ 1));
       __syncwarp();
       if (lane == 0) mbar_arrive(empty(s));
+      // slot a was last read by the MMAs of k-block kb - kSlots
+      if (kb >= C::kSlots) {
+        w = mbar_wait_bounded(afree(a), ((kb / C::kSlots) - 1) & 1, p.wait_limit_ns,
+                              abort_flag, p.status);
+        if (!__all_sync(0xFFFFFFFFu, w)) {
+          ok = false;
+          break;
+        }
+      }
       uint32_t u[32];
       unpack_word(lo.x, u + 0);
       unpack_word(lo.y, u + 4);
@@ -327,15 +339,11 @@ ternary_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_const
       unpack_word(hi.y, u + 20);
       unpack_word(hi.z, u + 24);
       unpack_word(hi.w, u + 28);
-      tc_st_32x32b_x32(tmem + lane_addr + C::kACol0 + s * 32, u);
+      tc_st_32x32b_x32(tmem + lane_addr + C::kACol0 + a * 32, u);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(afull(s));
-      if (++s == C::kStages) {
-        s = 0;
-        ph ^= 1u;
-      }
+      if (lane == 0) mbar_arrive(afull(a));
     }
     if (ok) {
       const bool w = mbar_wait_bounded(accfull, 0, p.wait_limit_ns, abort_flag, p.status);
@@ -524,6 +532,8 @@ cudaError_t launch_bn(const GemmCall& c, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_ternary_gemm(const GemmCall& c, cudaStream_t s) {
+  // prefill with room for the int8 weight codes: the CTA-pair GEMM
+  if (c.w8 != nullptr && prefill_ss_supported(c)) return launch_prefill_ss(c, c.w8, s);
   if (c.T <= 16) return launch_bn<16>(c, s);
   if (c.T <= 32) return launch_bn<32>(c, s);
   if (c.T <= 64) return launch_bn<64>(c, s);

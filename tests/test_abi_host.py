@@ -53,6 +53,10 @@ def test_workspace_sizes():
     assert L.mmf_forward_workspace_bytes(64, 1024, 1024) == 64 * 1024 + 256 + 256
     assert L.mmf_forward_workspace_bytes(3, 128, 128) == 512 + 256 + 256
     assert L.mmf_forward_workspace_bytes(0, 128, 128) == 0
+    # more than 128 tokens: also the weight codes expanded to int8, N x K
+    assert L.mmf_forward_workspace_bytes(300, 256, 512) == 300 * 256 + 2 * 1280 + 512 * 256
+    assert L.mmf_quantized_workspace_bytes(300, 256, 512) == 512 * 256
+    assert L.mmf_quantized_workspace_bytes(128, 256, 512) == 0
 
 
 A16 = 0x10000   # fake, aligned "device" addresses: never dereferenced by rejected calls
@@ -96,6 +100,11 @@ def test_glu_and_other_entry_points_reject_on_host():
     assert L.mmf_ternary_accumulate_i32(A16, 4, 256, A16, 256, A16 + 4, A16, 1 << 20,
                                         None) == ALIGN
     assert L.mmf_ternary_accumulate_i32(A16, 4, 256, A16, 256, A16, A16, 10, None) == WS
+    # a non-null workspace smaller than the query, or a size without a workspace
+    assert L.mmf_bitlinear_forward_quantized(A16, A16, A16, 300, 256, A16, A16, 512, 0, A16, 1,
+                                             A16, 1024, None) == WS
+    assert L.mmf_bitlinear_forward_quantized(A16, A16, A16, 300, 256, A16, A16, 512, 0, A16, 1,
+                                             None, 1024, None) == WS
     assert L.mmf_debug_wait_timeout_probe(10, None) == INVALID
     assert L.mmf_debug_wait_timeout_probe(10 ** 10, None) == INVALID
 

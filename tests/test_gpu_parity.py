@@ -100,8 +100,8 @@ def test_quantize_activations_zero_and_constant_rows():
 
 
 # ---------------------------------------------------------------------------- accumulator
-@pytest.mark.parametrize("T", [1, 7, 16, 17, 33, 64, 65, 100, 128, 129, 300, 517])
-@pytest.mark.parametrize("N,K", [(128, 128), (384, 1152)])
+@pytest.mark.parametrize("T", [1, 7, 16, 17, 33, 64, 65, 100, 128, 129, 300, 517, 1111])
+@pytest.mark.parametrize("N,K", [(128, 128), (384, 1152), (512, 640)])
 def test_accumulate_i32_bit_exact(T, N, K):
     q = synth.int8_codes(T, f"acc{T}", T, K)
     c = synth.ternary(N, f"acc{N}x{K}", N, K)
@@ -134,6 +134,11 @@ def test_accumulate_i32_extremes():
     # above the 256-token tile
     (8, 7040, 2560, np.float16, torch.float16),
     (300, 7040, 2560, np.float16, torch.float16),
+    # the persistent prefill kernel (T > 128): fp32 output, ragged last token tile, more
+    # tiles than SMs
+    (200, 640, 384, np.float16, torch.float32),
+    (1000, 1024, 1024, np.float16, torch.float16),
+    (1500, 512, 1280, np.float32, torch.float16),
 ])
 def test_forward_parity(T, K, N, dt, odt):
     x = synth.activations(T + N, f"fw{T}", T, K, dtype=dt)
@@ -145,16 +150,47 @@ def test_forward_parity(T, K, N, dt, odt):
     assert_out_close(y, y_ref)
 
 
-@pytest.mark.parametrize("T,K,I", [(1, 1024, 2816), (64, 1024, 2816), (8, 2048, 5632),
-                                   (130, 512, 192), (16, 2560, 7040)])
-def test_glu_forward_parity(T, K, I):
+@pytest.mark.parametrize("T,K,I,odt", [(1, 1024, 2816, torch.float16),
+                                       (64, 1024, 2816, torch.float16),
+                                       (8, 2048, 5632, torch.float16),
+                                       (130, 512, 192, torch.float16),
+                                       (16, 2560, 7040, torch.float16),
+                                       (300, 768, 320, torch.float32),
+                                       (777, 512, 640, torch.float16)])
+def test_glu_forward_parity(T, K, I, odt):
     x = synth.activations(T + I, f"glu{T}", T, K)
     W = synth.weights(K + I, f"glu{I}x{K}", 2 * I, K)
     Wp, beta = gpu_quantize_weights(W)
-    h = gpu_forward(x, Wp, beta, glu=True)
+    h = gpu_forward(x, Wp, beta, glu=True, out_dtype=odt)
     h_ref, beta_ref = oracle.bitlinear_forward(x, W, glu=True)
     assert beta == beta_ref
     assert_out_close(h, h_ref)
+
+
+@pytest.mark.parametrize("T,K,N,glu,odt", [(300, 1024, 512, False, torch.float16),
+                                            (257, 640, 768, True, torch.float16),
+                                            (1000, 512, 1024, False, torch.float32),
+                                            (513, 768, 512, True, torch.float32)])
+def test_quantized_forward_both_contractions_agree(T, K, N, glu, odt):
+    """From the same activation codes, the prefill contraction that expands the weights into a
+    workspace and the one that needs none give the same bits, and match the oracle."""
+    x = synth.activations(T + K, f"qf{T}", T, K)
+    W = synth.weights(N + K, f"qf{N}x{K}", N, K)
+    Wp, beta = gpu_quantize_weights(W)
+    A, gamma, rs = (to_dev(v) for v in gpu_act_quant(x))
+    Wpd, bd = to_dev(Wp), torch.tensor([beta], dtype=torch.float32, device=DEV)
+    n_out = N // 2 if glu else N
+    outs = []
+    for use_ws in (True, False):
+        y = torch.full((T, n_out), float("nan"), dtype=odt, device=DEV)
+        ws = mmf.workspace(mmf.mmf_quantized_workspace_bytes(T, K, N), DEV) if use_ws else None
+        mmf.mmf_bitlinear_forward_quantized(A, gamma, rs, Wpd, bd, N, glu, y, ws)
+        torch.cuda.synchronize()
+        outs.append(y.cpu())
+    assert torch.isfinite(outs[0]).all()
+    assert torch.equal(outs[0], outs[1])
+    y_ref = oracle_forward_from_parts(x, Wp, beta, K, glu=glu)
+    assert_out_close(outs[0].double().numpy(), y_ref)
 
 
 def test_forward_norm_weight_and_zero_rows():
