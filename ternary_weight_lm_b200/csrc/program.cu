@@ -112,6 +112,20 @@ struct PERec {
 static_assert(sizeof(PERec) == 64, "four 16-byte words");
 constexpr int kERecMax = 128;
 
+// What the producer, the unpack warps and the MMA warps need of a unit, flattened at plan time
+// and copied into shared memory at the start of a run (the first kSRecMax units of the CTA;
+// any further ones are read from the workspace).  A unit change then costs no dependent global
+// loads: with records read from the workspace, the producer stalled about a microsecond at
+// every unit boundary, which bounded the whole decode stream.
+struct PSRec {
+  const uint8_t* w;     // the unit's first 16 KB block of re-tiled weights
+  const int8_t* a;      // its input's tiled codes
+  int32_t nkb, kb0, level, pad;
+};
+static_assert(sizeof(PSRec) == 32, "two 16-byte words");
+template <int BN>
+constexpr int kSRecMax = BN <= 32 ? 256 : 64;
+
 struct PHeader {
   int32_t n_proj, n_in, n_levels, n_ctas, n_units, T, BN, n_tiles;
   float eps;
@@ -119,7 +133,7 @@ struct PHeader {
   uint32_t gen;         // init generation: every run passes the generation it was planned with
   int32_t pad;
   int64_t off_in, off_proj, off_units, off_ctaoff, off_wt, off_tilectr, off_levelctr, off_part;
-  int64_t off_erec;
+  int64_t off_erec, off_srec;
   int32_t in_begin[kMaxLevels + 1];
   int32_t qgroup[kMaxLevels];   // epilogue threads per input row in level L's quantisation
 };
@@ -134,12 +148,14 @@ struct PCfg {
   static constexpr int kTok = 8 * 64;             // per-token scale and code sum
   static constexpr int kOst = BN * 128 * 2;       // fp16 output staging [token][column]
   static constexpr int kERec = kERecMax * 64;     // staged epilogue records
-  static constexpr int kFixed = 1024 + 1024 + kXbuf + kTok + kOst + kERec + 64;
+  static constexpr int kSRec = kSRecMax<BN> * 32; // staged stream records
+  static constexpr int kFixed = 1024 + 1024 + kXbuf + kTok + kOst + kERec + kSRec + 64;
   static constexpr int kStagesFit = (227 * 1024 - 512 - kFixed) / kStage;
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
   static constexpr int kBar = (8 * (2 * kStages + kPGroups + 5) + 127) / 128 * 128;
-  static constexpr int kSmem = 1024 + kStages * kStage + kBar + kXbuf + kTok + kOst + kERec + 64;
-  static_assert(kStages >= 3, "pipeline depth");
+  static constexpr int kSmem =
+      1024 + kStages * kStage + kBar + kXbuf + kTok + kOst + kERec + kSRec + 64;
+  static_assert(kStages >= (BN <= 32 ? 6 : 4), "pipeline depth");
   static_assert(kBar <= 1024, "barrier area");
   static_assert(kSmem <= 227 * 1024 - 512, "shared memory");
   static_assert(kSmem >= 118 * 1024, "one CTA per SM");
@@ -495,6 +511,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
   int32_t* trs = reinterpret_cast<int32_t*>(tsc + 64);
   __half* ostage = reinterpret_cast<__half*>(trs + 64);
   uint4* s_erec = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(ostage) + C::kOst);
+  PSRec* s_srec = reinterpret_cast<PSRec*>(reinterpret_cast<uint8_t*>(s_erec) + C::kERec);
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ int s_flag;
@@ -559,8 +576,6 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
     return;
   }
   const PIn* ins = reinterpret_cast<const PIn*>(ws + H.off_in);
-  const PProj* projs = reinterpret_cast<const PProj*>(ws + H.off_proj);
-  const PUnit* units = reinterpret_cast<const PUnit*>(ws + H.off_units);
   const int32_t* ctaoff = reinterpret_cast<const int32_t*>(ws + H.off_ctaoff);
   unsigned* tilectr = reinterpret_cast<unsigned*>(const_cast<uint8_t*>(ws) + H.off_tilectr);
   unsigned* lvl = reinterpret_cast<unsigned*>(const_cast<uint8_t*>(ws) + H.off_levelctr);
@@ -571,6 +586,19 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
   const int nct = H.n_ctas;
   const int u_begin = ctaoff[blockIdx.x], u_end = ctaoff[blockIdx.x + 1];
   const int T = H.T;
+  const PSRec* g_srec = reinterpret_cast<const PSRec*>(ws + H.off_srec);
+  {
+    const int n4 = 2 * min(kSRecMax<BN>, u_end - u_begin);
+    const uint4* src = reinterpret_cast<const uint4*>(g_srec + u_begin);
+    for (int i = threadIdx.x; i < n4; i += kPThreads)
+      reinterpret_cast<uint4*>(s_srec)[i] = __ldg(src + i);
+  }
+  __syncthreads();
+  // unit ui of this CTA (u_begin <= ui < u_end)
+  auto srec = [&](int ui) -> PSRec {
+    const int j = ui - u_begin;
+    return j < kSRecMax<BN> ? s_srec[j] : g_srec[ui];
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -581,9 +609,6 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_a = l2_policy_evict_last();
-      // The unit records are read from the workspace once per unit into registers (the copy
-      // asm statements clobber memory, so a record read inside the stage loop would be
-      // re-fetched from L2 for every stage).
       struct Cur {
         int ui, k, nkb, kb0, level;
         const uint8_t* w;     // this unit's first weight block
@@ -593,13 +618,12 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         c.ui = ui;
         c.k = 0;
         if (ui >= u_end) return;
-        const PUnit u = units[ui];
-        const PProj pj = projs[u.proj];
-        c.nkb = u.nkb;
-        c.kb0 = u.kb0;
-        c.level = pj.level;
-        c.w = pj.Wt + (static_cast<int64_t>(u.tile) * pj.nst + u.kb0 / kPSub) * kPWStage;
-        c.a = ins[pj.in].A;
+        const PSRec r = srec(ui);
+        c.nkb = r.nkb;
+        c.kb0 = r.kb0;
+        c.level = r.level;
+        c.w = r.w;
+        c.a = r.a;
       };
       Cur wc, ac;
       load_cur(wc, u_begin);
@@ -617,38 +641,53 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         ac.k += kPSub;
         if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
       };
+      // Non-blocking loop: the activation copies of a stage wait for its level's codes, the
+      // weight copies only for a free stage, so the weights keep streaming (up to a full ring)
+      // while a level is being quantised.  A stretch with no progress at all is bounded.
+      uint64_t idle_since = 0;
       while (ok && ac.ui < u_end) {
-        // 1. the activation sub-tiles of every stage whose weights are already requested; at a
-        //    new level, first wait until its codes exist
+        bool progress = false;
+        // 1. activation sub-tiles of the stages whose weights are requested, once the level's
+        //    codes exist
         while (ai < wi) {
           if (ac.level > q_level) {
-            if (!grid_wait(lvl + 2 * ac.level, static_cast<unsigned>(nct), poison, limit_ns,
-                           status)) {
-              *abort_flag = 1;
-              ok = false;
-              break;
-            }
+            if (ld_acquire_u32(lvl + 2 * ac.level) < static_cast<unsigned>(nct)) break;
             fence_proxy_async_global();
             q_level = ac.level;
           }
           issue_act();
+          progress = true;
         }
-        if (!ok || wc.ui >= u_end) continue;
-        // 2. the packed weights of the next stage
-        const int st = static_cast<int>(wi % S);
-        if (wi >= S &&
-            !mbar_wait_bounded(empty(st), static_cast<uint32_t>(((wi / S) - 1) & 1), limit_ns,
-                               abort_flag, status)) {
-          ok = false;
-          break;
+        // 2. the packed weights of the next stage, if its ring slot is free
+        if (wc.ui < u_end) {
+          const int st = static_cast<int>(wi % S);
+          if (wi < static_cast<uint32_t>(S) ||
+              mbar_try_wait(empty(st), static_cast<uint32_t>(((wi / S) - 1) & 1))) {
+            const int nsub = min(kPSub, wc.nkb - wc.k);
+            mbar_arrive_expect_tx(full(st), kPWStage + nsub * C::kActSub);
+            bulk_load(smem_u32(s_w + st * kPWStage), wc.w + static_cast<int64_t>(wc.k / kPSub) * kPWStage,
+                      kPWStage, full(st), pol_w);
+            ++wi;
+            wc.k += kPSub;
+            if (wc.k >= wc.nkb) load_cur(wc, wc.ui + 1);
+            progress = true;
+          }
         }
-        const int nsub = min(kPSub, wc.nkb - wc.k);
-        mbar_arrive_expect_tx(full(st), kPWStage + nsub * C::kActSub);
-        bulk_load(smem_u32(s_w + st * kPWStage), wc.w + static_cast<int64_t>(wc.k / kPSub) * kPWStage,
-                  kPWStage, full(st), pol_w);
-        ++wi;
-        wc.k += kPSub;
-        if (wc.k >= wc.nkb) load_cur(wc, wc.ui + 1);
+        if (progress) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > limit_ns || ld_acquire_u32(poison) != 0u || *abort_flag) {
+            if (now - idle_since > limit_ns) {
+              atomicExch(poison, 1u);
+              atomicOr(status, kStatusTimeout);
+            }
+            *abort_flag = 1;
+            ok = false;
+          }
+        }
       }
       // Abort path: stages whose weights were requested but whose activations were not get
       // them now (the workspace buffer is valid memory), so that every started stage
@@ -670,10 +709,8 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
     uint32_t c = 0;                      // stage counter (32-bit: cheap % and /)
     bool ok = true;
     int n = 0;
-    int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
     for (int ui = u_begin; ui < u_end && ok; ++ui, ++n) {
-      const int nkb = next_nkb;
-      if (ui + 1 < u_end) next_nkb = units[ui + 1].nkb;   // overlaps this unit's MMAs
+      const int nkb = srec(ui).nkb;
       const int b = n & 1;
       const int ns = (nkb + kPSub - 1) / kPSub;
       // this warp's stages of the unit are s = first_s, first_s + 2, ... <= last_s
@@ -737,10 +774,8 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
     uint32_t c = 0;                      // stage counter (32-bit: cheap % and /)
     bool ok = true;
     int n = 0;
-    int next_nkb = u_begin < u_end ? units[u_begin].nkb : 0;
     for (int ui = u_begin; ui < u_end && ok; ++ui, ++n) {
-      const int nkb = next_nkb;
-      if (ui + 1 < u_end) next_nkb = units[ui + 1].nkb;   // overlaps this unit's MMAs
+      const int nkb = srec(ui).nkb;
       const int b = n & 1;
       if (n >= 2) {
         const bool w = mbar_wait_bounded(accempty(b), static_cast<uint32_t>(((n >> 1) - 1) & 1),
@@ -808,7 +843,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
     uint32_t c = 0;                      // stage counter (32-bit: cheap % and /)
     bool ok = true;
     for (int ui = u_begin; ui < u_end && ok; ++ui) {
-      const int nkb = units[ui].nkb;
+      const int nkb = srec(ui).nkb;
       for (int k = 0; k < nkb; k += kPSub, ++c) {
         if (static_cast<int>(c & 1) != set) continue;
         const int nsub = min(kPSub, nkb - k);
@@ -1107,6 +1142,7 @@ struct Plan {
   std::vector<PProj> projs;
   std::vector<PUnit> units;
   std::vector<PERec> erec;
+  std::vector<PSRec> srec;
   std::vector<int32_t> ctaoff;
   PHeader h;
   size_t bytes = 0;
@@ -1271,6 +1307,8 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
   off = al(off + P.units.size() * sizeof(PUnit), 256);
   h.off_erec = static_cast<int64_t>(off);
   off = al(off + P.units.size() * sizeof(PERec), 256);
+  h.off_srec = static_cast<int64_t>(off);
+  off = al(off + P.units.size() * sizeof(PSRec), 256);
   h.off_ctaoff = static_cast<int64_t>(off);
   off = al(off + P.ctaoff.size() * sizeof(int32_t), 256);
   h.off_tilectr = static_cast<int64_t>(off);
@@ -1299,6 +1337,18 @@ mmf_status build_plan(const mmf_projection* p, int n, int64_t T, float eps, uint
     off = al(off + static_cast<size_t>(q.N / 128) * q.nst * kPWStage, 256);
   }
   P.bytes = off;
+  P.srec.resize(P.units.size());
+  for (size_t i = 0; i < P.units.size(); ++i) {
+    const PUnit& u = P.units[i];
+    const PProj& q = P.projs[u.proj];
+    PSRec& r = P.srec[i];
+    r.w = q.Wt + (static_cast<int64_t>(u.tile) * q.nst + u.kb0 / kPSub) * kPWStage;
+    r.a = P.ins[q.in].A;
+    r.nkb = u.nkb;
+    r.kb0 = u.kb0;
+    r.level = q.level;
+    r.pad = 0;
+  }
   P.erec.resize(P.units.size());
   for (size_t i = 0; i < P.units.size(); ++i) {
     const PUnit& u = P.units[i];
@@ -1502,6 +1552,7 @@ MMF_EXPORT mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T
   std::memcpy(img.data() + P.h.off_proj, P.projs.data(), P.projs.size() * sizeof(PProj));
   std::memcpy(img.data() + P.h.off_units, P.units.data(), P.units.size() * sizeof(PUnit));
   std::memcpy(img.data() + P.h.off_erec, P.erec.data(), P.erec.size() * sizeof(PERec));
+  std::memcpy(img.data() + P.h.off_srec, P.srec.data(), P.srec.size() * sizeof(PSRec));
   std::memcpy(img.data() + P.h.off_ctaoff, P.ctaoff.data(), P.ctaoff.size() * sizeof(int32_t));
   // pageable source: the copy has consumed the host buffer when cudaMemcpyAsync returns
   if (cudaMemcpyAsync(ws, img.data(), img.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
