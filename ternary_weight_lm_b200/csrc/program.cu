@@ -43,8 +43,9 @@
 namespace mmf {
 namespace {
 
-// Warp roles: 0 TMA producer, 1 and 15 MMA issuers (even and odd stages; warp 1 alone for
-// 64-token tiles), 2-5 and 10-13 unpack (even and odd stages), 6-9 quantise + epilogue, 14 idle.
+// Warp roles: 0 and 14 TMA producers (weights, activation codes), 1 and 15 MMA issuers (even
+// and odd stages; warp 1 alone for 64-token tiles), 2-5 and 10-13 unpack (even and odd
+// stages), 6-9 quantise + epilogue.
 constexpr int kPThreads = 512;
 constexpr int kPEpi = 128;
 constexpr int kPEpiT0 = 192;               // first epilogue thread
@@ -53,9 +54,20 @@ constexpr int kPSub = 4;                   // sub-blocks per shared-memory stage
 constexpr int kPKS = kPKB * kPSub;         // K per stage (512)
 constexpr int kPWRow = kPKS / 4;           // packed bytes per weight row per stage: 128
 constexpr int kPWStage = 128 * kPWRow;     // 16 KB: one 128-byte line of each of 128 rows
-constexpr int kPSlots = 12;                // TMEM A slots of one sub-block each
-constexpr int kPGroups = kPSlots / kPSub;  // slot groups: stage counter c writes group c % 3
-constexpr int kPACol0 = 128;               // TMEM: accumulators at 0 and 64, slots from 128
+// TMEM: two accumulators (the next unit's MMAs run while the epilogue reads the other), then
+// A slots of one sub-block (32 columns) each.  Stage counter c writes slot group c % groups.
+// With 16-token tiles the accumulators take 64 columns.  (Stages of two sub-blocks, for a
+// deeper ring of seven slot groups, measured slower: a stage has a fixed cost.)
+template <int BN>
+constexpr int kPACol0 = BN <= 16 ? 64 : 128;
+template <int BN>
+constexpr int kPSlots = (512 - kPACol0<BN>) / 32;
+template <int BN>
+constexpr int kPGroups = kPSlots<BN> / kPSub;
+template <int BN>
+constexpr int kAccStride = BN <= 16 ? 32 : 64;    // TMEM columns per accumulator
+template <int BN>
+constexpr int kPartStride = BN <= 16 ? 16 : 32;   // second partial sum within an accumulator
 constexpr int kMaxLevels = 128;
 constexpr int kMaxProj = 1024;
 constexpr int kMaxSplit = 16;
@@ -63,7 +75,10 @@ constexpr int kMinSplitKb = 32;            // a split tile costs a few microseco
 constexpr uint64_t kPDrainNs = 2000000000ull;
 constexpr uint32_t kPlanMagic = 0x4d4d4650u;   // "PFMM"
 
-static_assert(kPACol0 + kPSlots * 32 == 512, "TMEM columns");
+static_assert(kPACol0<16> + kPSlots<16> * 32 == 512 && kPACol0<64> + kPSlots<64> * 32 == 512,
+              "TMEM columns");
+static_assert(2 * kAccStride<16> <= kPACol0<16> && 2 * kAccStride<64> <= kPACol0<64>,
+              "accumulators below the A slots");
 // Two partial accumulators per unit (even / odd sub-blocks) when they fit in the unit's 64
 // accumulator columns.
 template <int BN>
@@ -151,8 +166,8 @@ struct PCfg {
   static constexpr int kSRec = kSRecMax<BN> * 32; // staged stream records
   static constexpr int kFixed = 1024 + 1024 + kXbuf + kTok + kOst + kERec + kSRec + 64;
   static constexpr int kStagesFit = (227 * 1024 - 512 - kFixed) / kStage;
-  static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
-  static constexpr int kBar = (8 * (2 * kStages + kPGroups + 5) + 127) / 128 * 128;
+  static constexpr int kStages = kStagesFit < 16 ? kStagesFit : 16;
+  static constexpr int kBar = (8 * (2 * kStages + kPGroups<BN> + 5) + 127) / 128 * 128;
   static constexpr int kSmem =
       1024 + kStages * kStage + kBar + kXbuf + kTok + kOst + kERec + kSRec + 64;
   static_assert(kStages >= (BN <= 32 ? 6 : 4), "pipeline depth");
@@ -481,12 +496,12 @@ __device__ __forceinline__ void load_acc(uint32_t taddr, int32_t (&v)[CH]) {
   for (int j = 0; j < CH; ++j) v[j] = static_cast<int32_t>(u[j]);
 }
 
-template <int CH>
+template <int CH, int PS>
 __device__ __forceinline__ void load_acc_sum(uint32_t taddr, int mask, int32_t (&v)[CH]) {
-  load_acc<CH>(mask == 2 ? taddr + 32u : taddr, v);
+  load_acc<CH>(mask == 2 ? taddr + PS : taddr, v);
   if (mask == 3) {
     int32_t w[CH];
-    load_acc<CH>(taddr + 32u, w);
+    load_acc<CH>(taddr + PS, w);
 #pragma unroll
     for (int j = 0; j < CH; ++j) v[j] += w[j];
   }
@@ -530,9 +545,9 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
   auto full = [&](int st) { return smem_u32(bars + st); };
   auto empty = [&](int st) { return smem_u32(bars + S + st); };
   auto afull = [&](int gi) { return smem_u32(bars + 2 * S + gi); };
-  auto accfull = [&](int b) { return smem_u32(bars + 2 * S + kPGroups + b); };
-  auto accempty = [&](int b) { return smem_u32(bars + 2 * S + kPGroups + 2 + b); };
-  const uint32_t drainbar = smem_u32(bars + 2 * S + kPGroups + 4);
+  auto accfull = [&](int b) { return smem_u32(bars + 2 * S + kPGroups<BN> + b); };
+  auto accempty = [&](int b) { return smem_u32(bars + 2 * S + kPGroups<BN> + 2 + b); };
+  const uint32_t drainbar = smem_u32(bars + 2 * S + kPGroups<BN> + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -540,7 +555,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
       mbar_init(full(st), 1);
       mbar_init(empty(st), 1 + 4);
     }
-    for (int gi = 0; gi < kPGroups; ++gi) mbar_init(afull(gi), 4);
+    for (int gi = 0; gi < kPGroups<BN>; ++gi) mbar_init(afull(gi), 4);
     for (int b = 0; b < 2; ++b) {
       mbar_init(accfull(b), kTwoMma ? 2 : 1);   // one commit per MMA warp
       mbar_init(accempty(b), 4);
@@ -600,101 +615,59 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
     return j < kSRecMax<BN> ? s_srec[j] : g_srec[ui];
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 14) {
+    // ------------------------------------------------------------------ TMA producers
     // A stage is up to four k-blocks of one unit: the unit's 16 KB block of re-tiled weights
     // (one 128-byte line of each of the tile's 128 rows) and the stage's activation sub-tiles,
-    // each one contiguous bulk copy.  The weights run ahead of the activations (they do not
-    // depend on them), up to a full ring.
+    // each one contiguous bulk copy.  Two threads issue them: warp 0 the weights, warp 14 the
+    // activation codes.  Each waits for the stage to be free (empty) on its own, so the
+    // weights keep streaming, up to a full ring, while a level is being quantised, and the
+    // activation copies wait for their level's codes without holding the weights back.  (One
+    // thread issuing both took about 0.6 us per stage and bounded the decode stream.)  The
+    // weight thread sets the stage's expected bytes, both copies complete on full(s).
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
-      const uint64_t pol_a = l2_policy_evict_last();
-      struct Cur {
-        int ui, k, nkb, kb0, level;
-        const uint8_t* w;     // this unit's first weight block
-        const int8_t* a;      // the input's tiled codes
-      };
-      auto load_cur = [&](Cur& c, int ui) {
-        c.ui = ui;
-        c.k = 0;
-        if (ui >= u_end) return;
-        const PSRec r = srec(ui);
-        c.nkb = r.nkb;
-        c.kb0 = r.kb0;
-        c.level = r.level;
-        c.w = r.w;
-        c.a = r.a;
-      };
-      Cur wc, ac;
-      load_cur(wc, u_begin);
-      ac = wc;
-      uint32_t wi = 0, ai = 0;             // 32-bit: cheap % and /
-      int q_level = -1;
-      bool ok = true;
-      auto issue_act = [&]() {
-        const int st = static_cast<int>(ai % S);
-        const int nsub = min(kPSub, ac.nkb - ac.k);
-        // sub-blocks (kb0 + k) .. +nsub of the input, contiguous in its tiled codes
-        bulk_load(smem_u32(s_act + st * C::kAct), ac.a + static_cast<int64_t>(ac.kb0 + ac.k) * C::kActSub,
-                  static_cast<uint32_t>(nsub * C::kActSub), full(st), pol_a);
-        ++ai;
-        ac.k += kPSub;
-        if (ac.k >= ac.nkb) load_cur(ac, ac.ui + 1);
-      };
-      // Non-blocking loop: the activation copies of a stage wait for its level's codes, the
-      // weight copies only for a free stage, so the weights keep streaming (up to a full ring)
-      // while a level is being quantised.  A stretch with no progress at all is bounded.
-      uint64_t idle_since = 0;
-      while (ok && ac.ui < u_end) {
-        bool progress = false;
-        // 1. activation sub-tiles of the stages whose weights are requested, once the level's
-        //    codes exist
-        while (ai < wi) {
-          if (ac.level > q_level) {
-            if (ld_acquire_u32(lvl + 2 * ac.level) < static_cast<unsigned>(nct)) break;
-            fence_proxy_async_global();
-            q_level = ac.level;
-          }
-          issue_act();
-          progress = true;
-        }
-        // 2. the packed weights of the next stage, if its ring slot is free
-        if (wc.ui < u_end) {
-          const int st = static_cast<int>(wi % S);
-          if (wi < static_cast<uint32_t>(S) ||
-              mbar_try_wait(empty(st), static_cast<uint32_t>(((wi / S) - 1) & 1))) {
-            const int nsub = min(kPSub, wc.nkb - wc.k);
-            mbar_arrive_expect_tx(full(st), kPWStage + nsub * C::kActSub);
-            bulk_load(smem_u32(s_w + st * kPWStage), wc.w + static_cast<int64_t>(wc.k / kPSub) * kPWStage,
-                      kPWStage, full(st), pol_w);
-            ++wi;
-            wc.k += kPSub;
-            if (wc.k >= wc.nkb) load_cur(wc, wc.ui + 1);
-            progress = true;
-          }
-        }
-        if (progress) {
-          idle_since = 0;
+      const bool wts = warp == 0;
+      const uint64_t pol = wts ? l2_policy_evict_first() : l2_policy_evict_last();
+      int ui = u_begin, k = 0, q_level = -1;
+      PSRec r = {};
+      if (ui < u_end) r = srec(ui);
+      uint32_t i = 0;                      // stage counter (32-bit: cheap % and /)
+      while (ui < u_end) {
+        const int st = static_cast<int>(i % S);
+        if (i >= static_cast<uint32_t>(S) &&
+            !mbar_wait_bounded(empty(st), static_cast<uint32_t>(((i / S) - 1) & 1), limit_ns,
+                               abort_flag, status))
+          break;
+        const int nsub = min(kPSub, r.nkb - k);
+        if (wts) {
+          mbar_arrive_expect_tx(full(st), kPWStage + nsub * C::kActSub);
+          bulk_load(smem_u32(s_w + st * kPWStage), r.w + static_cast<int64_t>(k / kPSub) * kPWStage,
+                    kPWStage, full(st), pol);
         } else {
-          const uint64_t now = globaltimer_ns();
-          if (idle_since == 0) {
-            idle_since = now;
-          } else if (now - idle_since > limit_ns || ld_acquire_u32(poison) != 0u || *abort_flag) {
-            if (now - idle_since > limit_ns) {
-              atomicExch(poison, 1u);
-              atomicOr(status, kStatusTimeout);
+          if (r.level > q_level) {   // the level's codes exist once every CTA arrived
+            if (!grid_wait(lvl + 2 * r.level, static_cast<unsigned>(nct), poison, limit_ns,
+                           status)) {
+              *abort_flag = 1;
+              break;
             }
-            *abort_flag = 1;
-            ok = false;
+            fence_proxy_async_global();
+            q_level = r.level;
           }
+          // sub-blocks (kb0 + k) .. +nsub of the input, contiguous in its tiled codes
+          bulk_load(smem_u32(s_act + st * C::kAct), r.a + static_cast<int64_t>(r.kb0 + k) * C::kActSub,
+                    static_cast<uint32_t>(nsub * C::kActSub), full(st), pol);
+        }
+        ++i;
+        k += kPSub;
+        if (k >= r.nkb) {
+          k = 0;
+          if (++ui < u_end) r = srec(ui);
         }
       }
-      // Abort path: stages whose weights were requested but whose activations were not get
-      // them now (the workspace buffer is valid memory), so that every started stage
-      // completes; then wait until every copy this thread started has landed.
-      while (ai < wi && ac.ui < u_end) issue_act();
-      for (uint32_t i = wi > S ? wi - S : 0; i < wi; ++i)
-        mbar_wait_bounded(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1),
+      // Every copy this thread started lands before the block may exit (on the abort path a
+      // stage missing its other copy never completes; the bounded wait gives up on it).
+      for (uint32_t j = i > static_cast<uint32_t>(S) ? i - S : 0; j < i; ++j)
+        mbar_wait_bounded(full(static_cast<int>(j % S)), static_cast<uint32_t>((j / S) & 1),
                           kPDrainNs, nullptr, status);
     }
   } else if (kTwoMma && (warp == 1 || warp == 15)) {
@@ -716,7 +689,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
       // this warp's stages of the unit are s = first_s, first_s + 2, ... <= last_s
       const int first_s = static_cast<int>((c & 1) != static_cast<uint32_t>(mset));
       const int last_s = ns - 1 - static_cast<int>(((c + ns - 1) & 1) != static_cast<uint32_t>(mset));
-      const uint32_t d = tmem + static_cast<uint32_t>(b * 64 + mset * 32);
+      const uint32_t d = tmem + static_cast<uint32_t>(b * kAccStride<BN> + mset * kPartStride<BN>);
       if (n >= 2) {   // every MMA warp, even one with no stage here (see above)
         const bool w = mbar_wait_bounded(accempty(b), static_cast<uint32_t>(((n >> 1) - 1) & 1),
                                          limit_ns, abort_flag, status);
@@ -732,8 +705,8 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         if ((c & 1) != static_cast<uint32_t>(mset)) continue;
         const int nsub = min(kPSub, nkb - k);
         const int st = static_cast<int>(c % S);
-        const int gi = static_cast<int>(c % kPGroups);
-        const bool w = mbar_wait_bounded(afull(gi), static_cast<uint32_t>((c / kPGroups) & 1),
+        const int gi = static_cast<int>(c % kPGroups<BN>);
+        const bool w = mbar_wait_bounded(afull(gi), static_cast<uint32_t>((c / kPGroups<BN>) & 1),
                                          limit_ns, abort_flag, status);
         if (!__all_sync(0xFFFFFFFFu, w)) {
           ok = false;
@@ -742,7 +715,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         tc_fence_after();
         const int s_idx = k / kPSub;
         const uint64_t bst = bdesc0 + static_cast<uint64_t>((st * C::kAct) >> 4);
-        const uint32_t ast = tmem + kPACol0 + gi * kPSub * 32;
+        const uint32_t ast = tmem + kPACol0<BN> + gi * kPSub * 32;
         auto sub = [&](int i) {
           const uint64_t bd = bst + static_cast<uint64_t>((i * C::kActSub) >> 4);
           const uint32_t ad = ast + i * 32;
@@ -787,12 +760,12 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
       // sums, even sub-blocks at column 64b and odd ones at 64b + 32: consecutive MMAs into
       // different accumulators keep the tensor pipe busier than a chain on one (the epilogue
       // adds the two, exactly, in int32).
-      const uint32_t d = tmem + static_cast<uint32_t>(b * 64);
+      const uint32_t d = tmem + static_cast<uint32_t>(b * kAccStride<BN>);
       for (int k = 0; k < nkb; k += kPSub, ++c) {
         const int nsub = min(kPSub, nkb - k);
         const int st = static_cast<int>(c % S);
-        const int gi = static_cast<int>(c % kPGroups);
-        const bool w = mbar_wait_bounded(afull(gi), static_cast<uint32_t>((c / kPGroups) & 1),
+        const int gi = static_cast<int>(c % kPGroups<BN>);
+        const bool w = mbar_wait_bounded(afull(gi), static_cast<uint32_t>((c / kPGroups<BN>) & 1),
                                          limit_ns, abort_flag, status);
         if (!__all_sync(0xFFFFFFFFu, w)) {
           ok = false;
@@ -802,7 +775,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         // descriptor start address is in 16-byte units: a sub-tile is kActSub bytes, a 32-deep
         // k step is 32 bytes within the 128-byte swizzled rows
         const uint64_t bst = bdesc0 + static_cast<uint64_t>((st * C::kAct) >> 4);
-        const uint32_t ast = tmem + kPACol0 + gi * kPSub * 32;
+        const uint32_t ast = tmem + kPACol0<BN> + gi * kPSub * 32;
         auto sub = [&](int i) {
           const uint64_t bd = bst + static_cast<uint64_t>((i * C::kActSub) >> 4);
           const uint32_t ad = ast + i * 32;
@@ -848,11 +821,11 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         if (static_cast<int>(c & 1) != set) continue;
         const int nsub = min(kPSub, nkb - k);
         const int st = static_cast<int>(c % S);
-        const int gi = static_cast<int>(c % kPGroups);
+        const int gi = static_cast<int>(c % kPGroups<BN>);
         // Both conditions of this stage (its data landed; its slot group is free, see below)
         // are tested in one statement first; the bounded waits run only if one is not met.
-        const uint32_t cp = c - kPGroups;   // valid when c >= kPGroups
-        const bool both = c >= kPGroups && mbar_try_wait2(full(st), static_cast<uint32_t>((c / S) & 1),
+        const uint32_t cp = c - kPGroups<BN>;   // valid when c >= kPGroups
+        const bool both = c >= kPGroups<BN> && mbar_try_wait2(full(st), static_cast<uint32_t>((c / S) & 1),
                                                      empty(static_cast<int>(cp % S)),
                                                      static_cast<uint32_t>((cp / S) & 1));
         bool w = both || mbar_wait_bounded(full(st), static_cast<uint32_t>((c / S) & 1),
@@ -861,18 +834,19 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
           ok = false;
           break;
         }
-        // 128-byte swizzle: 16-byte chunk c of row r sits at chunk position c ^ (r mod 8)
+        // 128-byte swizzle: 16-byte chunk c of row r sits at chunk position c ^ (r mod 8), so
+        // the eight rows a quarter-warp reads hit eight bank groups
         const uint8_t* wrow = s_w + st * kPWStage + r * kPWRow;
-        uint4 ch[8];
+        uint4 ch[2 * kPSub];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc)
+        for (int cc = 0; cc < 2 * kPSub; ++cc)
           ch[cc] = *reinterpret_cast<const uint4*>(wrow + ((cc ^ (r & 7)) << 4));
         __syncwarp();
         if (lane == 0) mbar_arrive(empty(st));
         // slot group gi was last read by the MMAs of stage c - 3: their commit completed
         // empty((c - 3) % S).  (That barrier cannot have moved a further phase on: it needs
         // the arrivals for stage c - 3 + S, which come after this stage's.)
-        if (c >= kPGroups && !both) {
+        if (c >= kPGroups<BN> && !both) {
           w = mbar_wait_bounded(empty(static_cast<int>(cp % S)), static_cast<uint32_t>((cp / S) & 1),
                                 limit_ns, abort_flag, status);
           if (!__all_sync(0xFFFFFFFFu, w)) {
@@ -895,7 +869,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
             unpack_word4(hi.y, uu + 20);
             unpack_word4(hi.z, uu + 24);
             unpack_word4(hi.w, uu + 28);
-            tc_st_32x32b_x32(tmem + lane_addr + kPACol0 + (gi * kPSub + i) * 32, uu);
+            tc_st_32x32b_x32(tmem + lane_addr + kPACol0<BN> + (gi * kPSub + i) * 32, uu);
           }
         }
         tc_wait_st();
@@ -1015,7 +989,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
         ok = named_bar_and(1, kPEpi, __all_sync(0xFFFFFFFFu, w));   // also publishes tsc/trs
         if (!ok) break;
         tc_fence_after();
-        const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(b * 64);
+        const uint32_t dcol = tmem + lane_addr + static_cast<uint32_t>(b * kAccStride<BN>);
         // partial accumulators written for this unit: one per MMA warp (stage parity), both
         // when the unit has two or more stages
         const int ns_u = (u.nkb + kPSub - 1) / kPSub;
@@ -1025,7 +999,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
 #pragma unroll 1
           for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
             int32_t v[CH];
-            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), pmask, v);
+            load_acc_sum<CH, kPartStride<BN>>(dcol + static_cast<uint32_t>(c0), pmask, v);
             finalize_chunk<CH>(pj, u.tile, T, c0, v, r, tsc, trs, xbuf, ostage);
           }
           tc_fence_before();
@@ -1041,7 +1015,7 @@ program_kernel(const uint8_t* __restrict__ ws, uint32_t gen, unsigned* status, u
 #pragma unroll 1
           for (int c0 = 0; c0 < BN && c0 < T; c0 += CH) {
             int32_t v[CH];
-            load_acc_sum<CH>(dcol + static_cast<uint32_t>(c0), pmask, v);
+            load_acc_sum<CH, kPartStride<BN>>(dcol + static_cast<uint32_t>(c0), pmask, v);
 #pragma unroll
             for (int jj = 0; jj < CH; ++jj) atomicAdd(tacc + (c0 + jj) * 128 + r, v[jj]);
           }
@@ -1129,7 +1103,7 @@ __global__ void __launch_bounds__(128) retile_weights_kernel(const uint8_t* __re
   const uint8_t* src = Wp + static_cast<int64_t>(row) * row_bytes + st * kPWRow;
   uint8_t* dst = Wt + static_cast<int64_t>(blockIdx.x) * kPWStage + r * kPWRow;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
+  for (int c = 0; c < kPWRow / 16; ++c) {
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (st * kPWRow + c * 16 < row_bytes) v = *reinterpret_cast<const uint4*>(src + c * 16);
     *reinterpret_cast<uint4*>(dst + ((c ^ (r & 7)) << 4)) = v;
