@@ -38,6 +38,9 @@ def _L():
         lib.orc_silu_glu.argtypes = [P, I64, I64, P]
         lib.orc_bitlinear_forward.argtypes = [P, I64, I64, P, F, P, I64, ctypes.c_int, P]
         lib.orc_bitlinear_forward.restype = F
+        D = ctypes.c_double
+        lib.orc_mlgru_scan.argtypes = [P, P, I64, I64, P, P, P]
+        lib.orc_swish_gate_norm.argtypes = [P, P, I64, I64, P, D, P]
         _lib = lib
     return _lib
 
@@ -166,3 +169,41 @@ def bitlinear_forward(x, W, g=None, eps=1e-8, glu=False):
     beta = _L().orc_bitlinear_forward(_p(x), T, K, None if gg is None else _p(gg), eps, _p(W),
                                       N, 1 if glu else 0, _p(out))
     return out, np.float32(beta)
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a), dtype=np.float64)
+
+
+def mlgru_scan(I, F, h0=None):
+    """MLGRU recurrence h_t = sigmoid(F_t) h_{t-1} + (1 - sigmoid(F_t)) silu(I_t), in double.
+
+    ``I``, ``F``: [T, H]; ``h0``: [H] or None (zero).  Returns ``(h [T, H], hT [H])``.
+    """
+    I = _f64(I)
+    F = _f64(F)
+    T, H = I.shape
+    assert F.shape == (T, H)
+    hh = None if h0 is None else _f64(h0)
+    h = np.empty((T, H), dtype=np.float64)
+    hT = np.empty(H, dtype=np.float64)
+    _L().orc_mlgru_scan(_p(I), _p(F), T, H, None if hh is None else _p(hh), _p(h), _p(hT))
+    return h, hT
+
+
+def swish_gate_norm(h, G, w=None, eps=1e-8):
+    """FusedRMSNormSwishGate: h / sqrt(mean(h^2) + eps) * w * silu(G) per token, in double."""
+    h = _f64(h)
+    G = _f64(G)
+    T, H = h.shape
+    assert G.shape == (T, H)
+    ww = None if w is None else _f64(w)
+    o = np.empty((T, H), dtype=np.float64)
+    _L().orc_swish_gate_norm(_p(h), _p(G), T, H, None if ww is None else _p(ww), float(eps), _p(o))
+    return o
+
+
+def mlgru_forward(I, F, G, h0=None, w=None, eps=1e-8):
+    """Recurrence then the swish gate norm.  Returns ``(o [T, H] double, hT [H] double)``."""
+    h, hT = mlgru_scan(I, F, h0)
+    return swish_gate_norm(h, G, w, eps), hT

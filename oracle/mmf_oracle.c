@@ -21,6 +21,12 @@
  *       (one branch through SiLU, multiplied element-wise by the other).
  *  [P5] "量子化とは何か？MatMulというAIの計算やモデルサイズの最大のネック" (bluegarage, ja),
  *       section "MatMulとは具体的にどんな計算か" and its worked example "具体例".
+ *  [P4] again, section "Kernkomponenten: MLGRU und GLU", the MLGRU paragraph: the recurrence
+ *       runs token by token; each step takes the current token and the previous hidden state
+ *       and updates the state element-wise through gates, vectors of values between 0 and 1,
+ *       that weigh which parts of the previous state and of the current token carry on.
+ *  [P1] again: the gating of the attention side is FusedRMSNormSwishGate, and its output goes
+ *       through o_proj.
  *
  * Readings where the pages are silent (each is also listed with its reason in the design notes):
  *  - activations: per-token absmax to int8, s = 127/gamma, round half to even, clamp [-128,127];
@@ -32,6 +38,11 @@
  *  - dequantisation y = acc * (gamma/127) * beta and the GLU are evaluated in double;
  *  - GLU: the first half [0,I) of gate_proj's 2I outputs goes through SiLU, the second half is
  *    the multiplier.
+ *  - MLGRU (the pages give no formula): forget gate f = sigmoid(f_proj output), candidate
+ *    c = silu(i_proj output), h_t = f * h_{t-1} + (1 - f) * c, the state before the first token
+ *    given (zero by default); all in double.
+ *  - FusedRMSNormSwishGate: o = (h / sqrt(mean_j h_j^2 + eps)) * w * silu(g_proj output), the
+ *    mean over the H channels of one token, in double.
  *
  * Every decision that turns a float into an integer (an activation code, a weight code) is made
  * in IEEE single precision, the precision the GPU path uses for the same decision.
@@ -282,4 +293,48 @@ ORC_API float orc_bitlinear_forward(const float* x, int64_t T, int64_t K, const 
   free(c);
   free(acc);
   return beta;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* MLGRU recurrence ([P4] "Kernkomponenten: MLGRU und GLU", the MLGRU paragraph).  The pages    */
+/* describe it in words only: token by token, gates with values in (0, 1) weigh the previous    */
+/* hidden state against the current token, element-wise.  Reading taken: the forget gate       */
+/* f = sigmoid(F) keeps that share of the previous state and the rest, 1 - f, comes from the    */
+/* token's candidate c = silu(I):                                                                */
+/*     h_t = f_t * h_{t-1} + (1 - f_t) * c_t,    h_{-1} = h0 (zero when h0 is NULL).            */
+/* I, F: [T x H] row-major (the i_proj and f_proj outputs of T tokens).  h: [T x H], the state   */
+/* after each token.  hT: [H], the state after the last token (may be NULL).  Double throughout. */
+ORC_API void orc_mlgru_scan(const double* I, const double* F, int64_t T, int64_t H,
+                            const double* h0, double* h, double* hT) {
+  for (int64_t j = 0; j < H; ++j) {
+    double s = h0 ? h0[j] : 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+      double f = 1.0 / (1.0 + exp(-F[t * H + j]));
+      double z = I[t * H + j];
+      double c = z / (1.0 + exp(-z));
+      s = f * s + (1.0 - f) * c;
+      h[t * H + j] = s;
+    }
+    if (hT) hT[j] = s;
+  }
+}
+
+/* FusedRMSNormSwishGate ([P1] "HGRNBit という層構成を読む": the gate of the attention side, ahead */
+/* of o_proj).  Reading taken: an RMSNorm of the state over its H channels, scaled by the norm   */
+/* weight w (1 when NULL), times the swish (SiLU) of the g_proj output:                          */
+/*     o_tj = h_tj / sqrt(mean_j h_tj^2 + eps) * w_j * silu(G_tj).                              */
+/* h, G, o: [T x H] row-major.  Double throughout.                                               */
+ORC_API void orc_swish_gate_norm(const double* h, const double* G, int64_t T, int64_t H,
+                                 const double* w, double eps, double* o) {
+  for (int64_t t = 0; t < T; ++t) {
+    const double* hr = h + t * H;
+    double ss = 0.0;
+    for (int64_t j = 0; j < H; ++j) ss += hr[j] * hr[j];
+    double r = sqrt(ss / (double)H + eps);
+    for (int64_t j = 0; j < H; ++j) {
+      double g = G[t * H + j];
+      double sg = g / (1.0 + exp(-g));
+      o[t * H + j] = hr[j] / r * (w ? w[j] : 1.0) * sg;
+    }
+  }
 }

@@ -306,3 +306,102 @@ def test_forward_is_the_composition_of_its_steps():
     np.testing.assert_array_equal(y, oracle.dequant(acc, gamma, beta))
     h, _ = oracle.bitlinear_forward(x, W, g=g, glu=True)
     np.testing.assert_array_equal(h, oracle.silu_glu(y))
+
+
+# ----------------------------------------------------------------------------------------------
+# MLGRU recurrence and the swish gate norm.  The pages give the recurrence in words only (gates
+# in (0, 1) weigh the previous state against the current token), so the pins are the limits
+# that any such gate must reach, closed forms of the linear recurrence, and structure.
+# sigmoid and SiLU on the test side come from scipy's expit, not from the oracle.
+
+from scipy.special import expit  # noqa: E402
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def test_mlgru_closed_gate_takes_the_token():
+    # f -> 0 (F = -40 gives f < 5e-18, and 1 - f rounds to 1): the state is the candidate
+    I = _rand((7, 12), 1, 2.0)
+    F = np.full((7, 12), -40.0)
+    h, hT = oracle.mlgru_scan(I, F, h0=_rand(12, 2))
+    np.testing.assert_allclose(h, I * expit(I), rtol=1e-15, atol=1e-16)
+    np.testing.assert_array_equal(hT, h[-1])
+
+
+def test_mlgru_open_gate_keeps_the_state():
+    # f -> 1 (F = +40: f rounds to 1 in double): nothing of the tokens enters
+    h0 = _rand(9, 3)
+    h, hT = oracle.mlgru_scan(_rand((6, 9), 4, 3.0), np.full((6, 9), 40.0), h0=h0)
+    np.testing.assert_array_equal(h, np.broadcast_to(h0, (6, 9)))
+    np.testing.assert_array_equal(hT, h0)
+
+
+def test_mlgru_constant_inputs_geometric_series():
+    # constant gate f and candidate c from a zero state: h_t = c (1 - f^(t+1))
+    T, H = 40, 5
+    Fv = np.array([-2.0, -0.3, 0.0, 0.7, 2.5])
+    Iv = np.array([1.5, -0.8, 3.0, 0.25, -2.0])
+    h, _ = oracle.mlgru_scan(np.tile(Iv, (T, 1)), np.tile(Fv, (T, 1)))
+    f, c = expit(Fv), Iv * expit(Iv)
+    t = np.arange(1, T + 1)[:, None]
+    np.testing.assert_allclose(h, c * (1.0 - f ** t), rtol=1e-12, atol=1e-15)
+
+
+def test_mlgru_initial_state_enters_through_the_gate_product():
+    # the recurrence is affine in h0: h(h0) - h(0) = (prod_{s<=t} f_s) * h0
+    T, H = 30, 16
+    I, F, h0 = _rand((T, H), 5, 1.5), _rand((T, H), 6, 1.5), _rand(H, 7, 2.0)
+    h1, _ = oracle.mlgru_scan(I, F, h0)
+    h2, _ = oracle.mlgru_scan(I, F, None)
+    np.testing.assert_allclose(h1 - h2, np.cumprod(expit(F), axis=0) * h0, rtol=1e-9,
+                               atol=1e-13)
+
+
+def test_mlgru_split_sequence_carries_the_state():
+    # running the first part, then the rest from its final state, equals one run
+    T, H, t0 = 25, 11, 9
+    I, F, h0 = _rand((T, H), 8), _rand((T, H), 9), _rand(H, 10)
+    h, hT = oracle.mlgru_scan(I, F, h0)
+    ha, hTa = oracle.mlgru_scan(I[:t0], F[:t0], h0)
+    hb, hTb = oracle.mlgru_scan(I[t0:], F[t0:], hTa)
+    np.testing.assert_array_equal(np.concatenate([ha, hb]), h)
+    np.testing.assert_array_equal(hTb, hT)
+
+
+def test_mlgru_channels_are_independent():
+    # element-wise: permuting the channels permutes the states
+    I, F, h0 = _rand((8, 10), 11), _rand((8, 10), 12), _rand(10, 13)
+    perm = np.random.default_rng(14).permutation(10)
+    h, _ = oracle.mlgru_scan(I, F, h0)
+    hp, _ = oracle.mlgru_scan(I[:, perm], F[:, perm], h0[perm])
+    np.testing.assert_array_equal(hp, h[:, perm])
+
+
+def test_swish_gate_norm_unit_rms_with_linear_gate():
+    # G = 40: silu(G) = 40 to double precision, so o / (40 w) is h / r, whose mean square over
+    # the channels is ms / (ms + eps)
+    T, H = 6, 64
+    h, w = _rand((T, H), 15), 0.5 + np.abs(_rand(H, 16))
+    eps = 1e-3
+    o = oracle.swish_gate_norm(h, np.full((T, H), 40.0), w, eps)
+    ms = (h * h).mean(axis=1)
+    np.testing.assert_allclose(((o / (40.0 * w)) ** 2).mean(axis=1), ms / (ms + eps),
+                               rtol=1e-12)
+    # and the sign and proportions of h are kept channel by channel
+    np.testing.assert_allclose(o / (40.0 * w) * np.sqrt(ms + eps)[:, None], h, rtol=1e-12)
+
+
+def test_swish_gate_norm_scale_invariance_and_zero_gate():
+    T, H = 4, 32
+    h, G = _rand((T, H), 17), _rand((T, H), 18)
+    o1 = oracle.swish_gate_norm(h, G, None, 0.0)
+    o2 = oracle.swish_gate_norm(3.7 * h, G, None, 0.0)
+    np.testing.assert_allclose(o2, o1, rtol=1e-13)
+    assert np.all(oracle.swish_gate_norm(h, np.zeros((T, H)), None, 1e-8) == 0.0)
+    # the gate is SiLU, odd around its own definition: silu(g) - silu(-g) = g
+    op = oracle.swish_gate_norm(h, G, None, 1e-8)
+    om = oracle.swish_gate_norm(h, -G, None, 1e-8)
+    r = np.sqrt((h * h).mean(axis=1) + 1e-8)[:, None]
+    np.testing.assert_allclose((op - om) * r / h, G, rtol=1e-10, atol=1e-12)
