@@ -204,6 +204,43 @@ mmf_status mmf_program_init(const mmf_projection* p, int n, int64_t T, float eps
  * Calls on one workspace must not overlap. */
 mmf_status mmf_program_run(void* ws, void* stream);
 
+/* ---- MLGRU recurrence + FusedRMSNormSwishGate ----------------------------------------------
+ * [P4] "MatMul-freie LLMs: Zentrale Konzepte erklärt", section "Kernkomponenten: MLGRU und GLU",
+ * the MLGRU paragraph: token by token, element-wise gates with values between 0 and 1 weigh
+ * the previous hidden state against the current token.  [P1] section "HGRNBit という層構成を読む":
+ * the attention side gates through FusedRMSNormSwishGate ahead of o_proj.  The pages give no
+ * formula; the library computes, for the i/f/g projection outputs I, F, G [T x H] and j < H:
+ *   f_tj = sigmoid(F_tj),  c_tj = silu(I_tj),  h_tj = f_tj * h_(t-1)j + (1 - f_tj) * c_tj
+ *   o_tj = h_tj / sqrt(mean_j h_tj^2 + eps) * w_j * silu(G_tj)
+ * with h before the first token = h0 (zero when NULL), in float (exp and reciprocals through
+ * the fast intrinsics: relative error a few 1e-6 before the output's own rounding).  Tokens are
+ * scanned in chunks of 64; chunk boundaries change only the rounding order of h.
+ *
+ * Shapes: 1 <= T <= 16777216; H a multiple of 256, 256 <= H <= 4096.  I, F, G, o: row-major,
+ * 16-byte aligned, all of dtype xdt (I/F/G) and odt (o).  h0, hT, norm_w: [H] fp32 (may be
+ * NULL), 16-byte aligned.  ws: mmf_mlgru_workspace_bytes(T, H) bytes, 256-byte aligned (NULL
+ * with ws_bytes 0 when that is 0, i.e. T <= 64).  Errors as for the forward; a workspace that
+ * is missing or too small: MMF_ERR_WORKSPACE.  Asynchronous on `stream`. */
+size_t mmf_mlgru_workspace_bytes(int64_t T, int64_t H);
+
+mmf_status mmf_mlgru_forward(const void* I, const void* F, const void* G, mmf_dtype xdt,
+                             int64_t T, int64_t H, const float* h0, const float* norm_w,
+                             float eps, void* o, mmf_dtype odt, float* hT, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* The same recurrence and gate, fused with o_proj's activation pre-pass: instead of o it
+ * writes what mmf_quantize_activations(o16, MMF_F16, T, H, oproj_norm_w, oproj_eps, A, gamma,
+ * rowsum) would write for o16 = o rounded to fp16 (A [T x H] int8 row-major, gamma [T],
+ * rowsum [T] or NULL), ready for mmf_bitlinear_forward_quantized with K = H.  The sum of
+ * squares of a row is added in another order, so in rare rows its last bit, and with it a
+ * code, can differ from the separate pre-pass. */
+mmf_status mmf_mlgru_forward_quantized(const void* I, const void* F, const void* G,
+                                       mmf_dtype xdt, int64_t T, int64_t H, const float* h0,
+                                       const float* norm_w, float eps,
+                                       const float* oproj_norm_w, float oproj_eps, int8_t* A,
+                                       float* gamma, int32_t* rowsum, float* hT, void* ws,
+                                       size_t ws_bytes, void* stream);
+
 /* ---- forward without any allocation ------------------------------------------------------ */
 
 /* The pages have no counterpart to this entry point; it serves callers that cannot call

@@ -23,6 +23,8 @@ __all__ = [
     "mmf_debug_wait_timeout_probe", "mmf_status_string", "mmf_version",
     "mmf_program_workspace_bytes", "mmf_program_init", "mmf_program_run", "Projection",
     "Program", "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
+    "mmf_mlgru_workspace_bytes", "mmf_mlgru_forward", "mmf_mlgru_forward_quantized",
+    "mlgru_forward",
     "MMF_F32", "MMF_F16", "STATUS",
 ]
 
@@ -77,6 +79,10 @@ def lib():
                                                 I),
             "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
             "mmf_bitlinear_forward_noalloc": ([P, I, I64, I64, P, F, P, P, I64, P, I, P], I),
+            "mmf_mlgru_workspace_bytes": ([I64, I64], SZ),
+            "mmf_mlgru_forward": ([P, P, P, I, I64, I64, P, P, F, P, I, P, P, SZ, P], I),
+            "mmf_mlgru_forward_quantized": ([P, P, P, I, I64, I64, P, P, F, P, F, P, P, P, P, P,
+                                             SZ, P], I),
             "mmf_program_workspace_bytes": ([P, I, I64], SZ),
             "mmf_program_init": ([P, I, I64, F, P, SZ, P], I),
             "mmf_program_run": ([P, P], I),
@@ -200,6 +206,34 @@ def mmf_bitlinear_forward_noalloc(x, norm_w, eps, Wp, beta, N, y, stream=None):
         _dt(y), _stream(stream)))
 
 
+def mmf_mlgru_workspace_bytes(T, H):
+    return lib().mmf_mlgru_workspace_bytes(T, H)
+
+
+def _ws(ws):
+    return (None, 0) if ws is None else (_ptr(ws), _nbytes(ws))
+
+
+def mmf_mlgru_forward(I, F, G, h0, norm_w, eps, o, hT=None, ws=None, stream=None):
+    """MLGRU recurrence + swish gate norm (include/mmf.h): o [T, H] from I, F, G [T, H]."""
+    T, H = I.shape
+    wp, wn = _ws(ws)
+    _check("mmf_mlgru_forward", lib().mmf_mlgru_forward(
+        _ptr(I), _ptr(F), _ptr(G), _dt(I), T, H, _ptr(h0), _ptr(norm_w), float(eps), _ptr(o),
+        _dt(o), _ptr(hT), wp, wn, _stream(stream)))
+
+
+def mmf_mlgru_forward_quantized(I, F, G, h0, norm_w, eps, oproj_norm_w, oproj_eps, A, gamma,
+                                rowsum=None, hT=None, ws=None, stream=None):
+    """The same, writing o_proj's int8 codes, gamma and code sums instead of o."""
+    T, H = I.shape
+    wp, wn = _ws(ws)
+    _check("mmf_mlgru_forward_quantized", lib().mmf_mlgru_forward_quantized(
+        _ptr(I), _ptr(F), _ptr(G), _dt(I), T, H, _ptr(h0), _ptr(norm_w), float(eps),
+        _ptr(oproj_norm_w), float(oproj_eps), _ptr(A), _ptr(gamma), _ptr(rowsum), _ptr(hT), wp,
+        wn, _stream(stream)))
+
+
 def _proj_array(projs):
     arr = (Projection * len(projs))()
     for i, p in enumerate(projs):
@@ -288,6 +322,20 @@ def bitlinear_forward(x, Wp, beta, norm_w=None, eps=1e-8, out_dtype=None, ws=Non
         ws = workspace(mmf_forward_workspace_bytes(T, K, N), x.device)
     mmf_bitlinear_forward(x, norm_w, eps, Wp, beta, N, y, ws, stream)
     return y
+
+
+def mlgru_forward(I, F, G, h0=None, norm_w=None, eps=1e-8, out_dtype=None, hT=None, ws=None,
+                  stream=None):
+    """o [T, H] of the MLGRU recurrence and swish gate norm; hT (optional [H] fp32) receives
+    the state after the last token."""
+    import torch
+    T, H = I.shape
+    o = torch.empty((T, H), dtype=out_dtype or I.dtype, device=I.device)
+    need = mmf_mlgru_workspace_bytes(T, H)
+    if ws is None and need > 0:
+        ws = workspace(need, I.device)
+    mmf_mlgru_forward(I, F, G, h0, norm_w, eps, o, hT, ws, stream)
+    return o
 
 
 def bitlinear_glu_forward(x, Wp, beta, norm_w=None, eps=1e-8, out_dtype=None, ws=None,

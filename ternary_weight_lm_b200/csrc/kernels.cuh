@@ -58,6 +58,34 @@ size_t prefill_w8_bytes(int64_t N, int64_t K);
 bool prefill_ss_supported(const GemmCall& c);
 cudaError_t launch_prefill_ss(const GemmCall& c, int8_t* w8, cudaStream_t s);
 
+// MLGRU recurrence + swish gate norm over T tokens (chunked scan, three launches; one when
+// T <= 64).  amap/bmap/carry: workspace arrays of [chunks x H] floats (mlgru_ws_bytes).  With A
+// set, o_proj's codes/gamma/rowsum are written instead of o.
+struct MlgruCall {
+  const void* I;
+  const void* F;
+  const void* G;
+  int xdt;
+  int64_t T;
+  int H;
+  const float* h0;
+  const float* norm_w;
+  float eps;
+  void* o;
+  int odt;
+  const float* q_norm_w;
+  float q_eps;
+  int8_t* A;
+  float* gamma;
+  int32_t* rowsum;
+  float* hT;
+  float* amap;
+  float* bmap;
+  float* carry;
+};
+size_t mlgru_ws_bytes(int64_t T, int64_t H);
+cudaError_t launch_mlgru(const MlgruCall& c, cudaStream_t s);
+
 // Device address of the library's status word on the current device (nullptr on failure).
 unsigned* device_status_word();
 

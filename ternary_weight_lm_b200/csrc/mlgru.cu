@@ -1,0 +1,437 @@
+// MLGRU recurrence and FusedRMSNormSwishGate over T tokens, with o_proj's activation
+// quantisation fused into the output pass on request.
+//
+// What it computes (the pages describe the recurrence in words only, "MatMul-freie LLMs:
+// Zentrale Konzepte erklärt", section "Kernkomponenten: MLGRU und GLU": token by token, gates
+// with values between 0 and 1 weigh the previous hidden state against the current token,
+// element-wise; the gate of the attention side is FusedRMSNormSwishGate, ahead of o_proj,
+// "matmulfreellm 評価", section "HGRNBit という層構成を読む").  Per channel j < H:
+//     f = sigmoid(F_tj),  c = silu(I_tj),  h_tj = f * h_(t-1)j + (1 - f) * c
+//     o_tj = h_tj / sqrt(mean_j h_tj^2 + eps) * w_j * silu(G_tj)
+// with h before the first token given (zero by default).  I, F, G are the i_proj, f_proj and
+// g_proj outputs [T x H].
+//
+// The recurrence is a chain of affine maps h -> a h + b, which compose associatively, so the T
+// tokens are cut into chunks of kChunk and scanned in three launches:
+//   (A) chunk maps: every (chunk, 8 channels) thread composes its chunk's maps, (a, b);
+//   (B) carries: one warp per channel scans the chunk maps (shuffles over 32 chunks at a time)
+//       into the state entering each chunk;
+//   (C) outputs: one CTA per chunk and all H channels (one 16-byte vector of 8 channels per
+//       thread) runs the chunk from its carry and finishes every token's gate norm with a
+//       block reduction; it writes o in fp16/fp32, or, fused, o_proj's int8 codes, gamma and
+//       code sums computed from o rounded to fp16, the same arithmetic as the activation
+//       pre-pass applied to that fp16 o.
+// With T <= kChunk, (C) alone runs from the initial state.
+//
+// Rooflines: HBM-bound.  (A) reads I and F, (C) reads I, F and G and writes o: 12 bytes per
+// element in fp16 against the 8 of one pass.  The exponentials and reciprocals go through the
+// special function units (16 per SM per clock); f and sigmoid(I) share one reciprocal, so (A)
+// takes 3 and (C) 5 such operations per element.
+#include <cuda_fp16.h>
+
+#include "kernels.cuh"
+
+namespace mmf {
+namespace {
+
+constexpr int kChunk = 64;       // tokens per chunk
+constexpr int kAThreads = 128;   // threads per CTA of the chunk-map kernel
+constexpr int kTB = 4;           // tokens per block reduction in the output kernel
+// |x| cap before exp.  At +-40 a gate is within 5e-18 of its limit, and (1 + e1)(1 + e2) stays
+// below 2^116: __fdividef(1, y) returns 0 for y above 2^126, which with a cap of 80 zeroed
+// gates of ~1e-3 whenever the other exponential was near its cap.
+constexpr float kClamp = 40.0f;
+
+// 8 channels of one row as floats: one 16-byte fp16 vector, or two of fp32.
+template <int XDT>
+__device__ __forceinline__ void load8(const void* base, int64_t off, float (&v)[8]) {
+  if (XDT == kInF16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const __half*>(base) + off);
+    const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
+    const float4 b =
+        *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// One token's map for one channel: h -> f h + (1 - f) c.  With e1 = exp(-F), e2 = exp(-I):
+// f = 1/(1+e1) and sigmoid(I) = 1/(1+e2) come from one reciprocal of (1+e1)(1+e2), and
+// 1 - f = e1 f without cancellation.  Inputs are capped at +-kClamp first.
+__device__ __forceinline__ void token_map(float F, float I, float& f, float& u) {
+  const float e1 = __expf(-fminf(fmaxf(F, -kClamp), kClamp));
+  const float e2 = __expf(-fminf(fmaxf(I, -kClamp), kClamp));
+  const float d1 = 1.0f + e1, d2 = 1.0f + e2;
+  const float r = __fdividef(1.0f, d1 * d2);
+  f = r * d2;
+  const float sI = r * d1;
+  u = (e1 * f) * (I * sI);          // (1 - f) * silu(I)
+}
+
+__device__ __forceinline__ float silu_f(float g) {
+  const float e = __expf(-fminf(fmaxf(g, -kClamp), kClamp));
+  return g * __fdividef(1.0f, 1.0f + e);
+}
+
+// ------------------------------------------------------------------------------- (A) chunk maps
+template <int XDT>
+__global__ void __launch_bounds__(kAThreads) mlgru_chunk_kernel(const void* I, const void* F,
+                                                                int64_t T, int H, float* Amap,
+                                                                float* Bmap) {
+  const int chunk = blockIdx.x;
+  const int v = blockIdx.y * kAThreads + threadIdx.x;    // vector of channels 8v .. 8v+7
+  if (8 * v >= H) return;
+  const int64_t t0 = static_cast<int64_t>(chunk) * kChunk;
+  const int nt = static_cast<int>(T - t0 < kChunk ? T - t0 : kChunk);
+  float a[8], b[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    a[k] = 1.0f;
+    b[k] = 0.0f;
+  }
+  const int64_t base = t0 * H + 8 * v;
+  int t = 0;
+  // four tokens' loads in flight before their maps are applied
+  for (; t + 4 <= nt; t += 4) {
+    float iv[4][8], fv[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      load8<XDT>(I, base + static_cast<int64_t>(t + u) * H, iv[u]);
+      load8<XDT>(F, base + static_cast<int64_t>(t + u) * H, fv[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float f, w;
+        token_map(fv[u][k], iv[u][k], f, w);
+        a[k] *= f;
+        b[k] = fmaf(f, b[k], w);
+      }
+  }
+  for (; t < nt; ++t) {
+    float iv[8], fv[8];
+    load8<XDT>(I, base + static_cast<int64_t>(t) * H, iv);
+    load8<XDT>(F, base + static_cast<int64_t>(t) * H, fv);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      float f, w;
+      token_map(fv[k], iv[k], f, w);
+      a[k] *= f;
+      b[k] = fmaf(f, b[k], w);
+    }
+  }
+  float4* ao = reinterpret_cast<float4*>(Amap + static_cast<int64_t>(chunk) * H + 8 * v);
+  float4* bo = reinterpret_cast<float4*>(Bmap + static_cast<int64_t>(chunk) * H + 8 * v);
+  ao[0] = make_float4(a[0], a[1], a[2], a[3]);
+  ao[1] = make_float4(a[4], a[5], a[6], a[7]);
+  bo[0] = make_float4(b[0], b[1], b[2], b[3]);
+  bo[1] = make_float4(b[4], b[5], b[6], b[7]);
+}
+
+// ------------------------------------------------------------------------------- (B) carries
+// One warp per channel.  Lane l takes chunk k0 + l; an inclusive shuffle scan composes the maps
+// of chunks k0 .. k0 + l (later map applied after the earlier one: (a, b) after (a', b') is
+// (a a', a b' + b)); the carry into chunk k is the exclusive composite applied to the state s
+// entering chunk k0.  Lanes past the last chunk hold the identity map.
+__global__ void __launch_bounds__(128) mlgru_carry_kernel(const float* Amap, const float* Bmap,
+                                                          const float* h0, int nch, int H,
+                                                          float* carry) {
+  const int j = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= H) return;
+  float s = h0 != nullptr ? h0[j] : 0.0f;
+  for (int k0 = 0; k0 < nch; k0 += 32) {
+    const int k = k0 + lane;
+    float a = 1.0f, b = 0.0f;
+    if (k < nch) {
+      a = Amap[static_cast<int64_t>(k) * H + j];
+      b = Bmap[static_cast<int64_t>(k) * H + j];
+    }
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const float ap = __shfl_up_sync(0xffffffffu, a, d);
+      const float bp = __shfl_up_sync(0xffffffffu, b, d);
+      if (lane >= d) {
+        b = fmaf(a, bp, b);
+        a *= ap;
+      }
+    }
+    float ae = __shfl_up_sync(0xffffffffu, a, 1);
+    float be = __shfl_up_sync(0xffffffffu, b, 1);
+    if (lane == 0) {
+      ae = 1.0f;
+      be = 0.0f;
+    }
+    if (k < nch) carry[static_cast<int64_t>(k) * H + j] = fmaf(ae, s, be);
+    const float al = __shfl_sync(0xffffffffu, a, 31);
+    const float bl = __shfl_sync(0xffffffffu, b, 31);
+    s = fmaf(al, s, bl);
+  }
+}
+
+// ------------------------------------------------------------------------------- (C) outputs
+__device__ __forceinline__ int code_s8(float y) {
+  int q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(q) : "f"(y));
+  return q;
+}
+
+__device__ __forceinline__ uint32_t pack4(int q0, int q1, int q2, int q3) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(q0), static_cast<uint32_t>(q1), 0x0040);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(q2), static_cast<uint32_t>(q3), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+struct OutArgs {
+  const void* I;
+  const void* F;
+  const void* G;
+  int64_t T;
+  int H;
+  const float* carry;    // [nch x H] state entering each chunk, or (one chunk) h0, or nullptr
+  const float* norm_w;   // gate norm weight [H] or nullptr
+  float eps;
+  void* o;               // [T x H] fp16 / fp32 (plain mode)
+  int odt;               // kInF16 / kInF32
+  const float* q_norm_w; // o_proj norm weight [H] or nullptr (fused mode)
+  float q_eps;
+  int8_t* A;             // [T x H] o_proj codes, gamma [T], rowsum [T] (fused mode)
+  float* gamma;
+  int32_t* rowsum;
+  float* hT;             // [H] final state or nullptr
+};
+
+// Block reduction of kTB per-thread values of type V (sum or max): every thread gets the
+// totals.  red: 2 buffers x kTB x 32 warps; the buffer alternates, so one barrier per round.
+template <typename V, bool MAX>
+__device__ __forceinline__ void block_reduce(V (&x)[kTB], V* red, int& buf, int nwarps) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int u = 0; u < kTB; ++u) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const V y = __shfl_xor_sync(0xffffffffu, x[u], o);
+      x[u] = MAX ? (y > x[u] ? y : x[u]) : x[u] + y;
+    }
+  }
+  V* r = red + buf * (kTB * 32);
+  if (lane == 0)
+#pragma unroll
+    for (int u = 0; u < kTB; ++u) r[u * 32 + warp] = x[u];
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kTB; ++u) {
+    V acc = r[u * 32];
+    for (int w = 1; w < nwarps; ++w) {
+      const V y = r[u * 32 + w];
+      acc = MAX ? (y > acc ? y : acc) : acc + y;
+    }
+    x[u] = acc;
+  }
+  buf ^= 1;
+}
+
+template <int XDT, bool QUANT>
+__global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
+  __shared__ float red_f[2 * kTB * 32];
+  __shared__ double red_d[2 * kTB * 32];
+  __shared__ int red_i[2 * kTB * 32];
+  const int chunk = blockIdx.x;
+  const int v = threadIdx.x;                 // channels 8v .. 8v+7
+  const int H = p.H;
+  const int nwarps = blockDim.x >> 5;
+  const int64_t t0 = static_cast<int64_t>(chunk) * kChunk;
+  const int nt = static_cast<int>(p.T - t0 < kChunk ? p.T - t0 : kChunk);
+  float s[8], w[8], qw[8];
+  {
+    const float* c = p.carry != nullptr ? p.carry + static_cast<int64_t>(chunk) * H : nullptr;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      s[k] = c != nullptr ? c[8 * v + k] : 0.0f;
+      w[k] = p.norm_w != nullptr ? p.norm_w[8 * v + k] : 1.0f;
+      qw[k] = (QUANT && p.q_norm_w != nullptr) ? p.q_norm_w[8 * v + k] : 1.0f;
+    }
+  }
+  int fb = 0, db = 0, ib = 0;
+  const float invH = 1.0f / static_cast<float>(H);
+  for (int tb = 0; tb < nt; tb += kTB) {
+    float hv[kTB][8], gv[kTB][8];
+    float ss[kTB];
+#pragma unroll
+    for (int u = 0; u < kTB; ++u) {
+      ss[u] = 0.0f;
+      if (tb + u < nt) {
+        const int64_t off = (t0 + tb + u) * H + 8 * v;
+        float iv[8], fv[8];
+        load8<XDT>(p.I, off, iv);
+        load8<XDT>(p.F, off, fv);
+        load8<XDT>(p.G, off, gv[u]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float f, uu;
+          token_map(fv[k], iv[k], f, uu);
+          s[k] = fmaf(f, s[k], uu);
+          hv[u][k] = s[k];
+          ss[u] = fmaf(s[k], s[k], ss[u]);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          hv[u][k] = 0.0f;
+          gv[u][k] = 0.0f;
+        }
+      }
+    }
+    block_reduce<float, false>(ss, red_f, fb, nwarps);
+    // o = h / r * w * silu(g), r = sqrt(mean h^2 + eps)
+#pragma unroll
+    for (int u = 0; u < kTB; ++u) {
+      const float inv = __fdiv_rn(1.0f, __fsqrt_rn(fmaf(ss[u], invH, p.eps)));
+#pragma unroll
+      for (int k = 0; k < 8; ++k) hv[u][k] = hv[u][k] * inv * w[k] * silu_f(gv[u][k]);
+    }
+    if (!QUANT) {
+#pragma unroll
+      for (int u = 0; u < kTB; ++u) {
+        if (tb + u >= nt) break;
+        const int64_t off = (t0 + tb + u) * H + 8 * v;
+        if (p.odt == kInF16) {
+          uint4 pk;
+          __half2* h2 = reinterpret_cast<__half2*>(&pk);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) h2[i] = __floats2half2_rn(hv[u][2 * i], hv[u][2 * i + 1]);
+          *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.o) + off) = pk;
+        } else {
+          float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + off);
+          d[0] = make_float4(hv[u][0], hv[u][1], hv[u][2], hv[u][3]);
+          d[1] = make_float4(hv[u][4], hv[u][5], hv[u][6], hv[u][7]);
+        }
+      }
+    } else {
+      // o_proj's pre-pass on o rounded to fp16: mean of squares in double, rounded once;
+      // inv = 1/sqrt(ms + eps); xhat = (x * inv) * g; gamma = max|xhat| floored at 1e-5;
+      // q = rne(xhat * (127/gamma)), saturated.  Without a norm weight gamma = max|x| * inv.
+      double sd[kTB];
+      float mx[kTB];
+#pragma unroll
+      for (int u = 0; u < kTB; ++u) {
+        sd[u] = 0.0;
+        mx[u] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          hv[u][k] = __half2float(__float2half_rn(hv[u][k]));
+          const double dx = static_cast<double>(hv[u][k]);
+          sd[u] = fma(dx, dx, sd[u]);
+          mx[u] = fmaxf(mx[u], fabsf(hv[u][k]));
+        }
+      }
+      block_reduce<double, false>(sd, red_d, db, nwarps);
+      float inv[kTB], amax[kTB];
+#pragma unroll
+      for (int u = 0; u < kTB; ++u) {
+        const float ms = __double2float_rn(__ddiv_rn(sd[u], static_cast<double>(H)));
+        inv[u] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.q_eps)));
+        if (p.q_norm_w == nullptr) {
+          amax[u] = mx[u];
+        } else {
+          amax[u] = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            amax[u] = fmaxf(amax[u], fabsf(__fmul_rn(__fmul_rn(hv[u][k], inv[u]), qw[k])));
+        }
+      }
+      block_reduce<float, true>(amax, red_f, fb, nwarps);
+      int rs[kTB];
+#pragma unroll
+      for (int u = 0; u < kTB; ++u) {
+        const float gm = fmaxf(p.q_norm_w == nullptr ? __fmul_rn(amax[u], inv[u]) : amax[u],
+                               1e-5f);
+        const float sc = __fdiv_rn(127.0f, gm);
+        int q[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          float xh = __fmul_rn(hv[u][k], inv[u]);
+          if (p.q_norm_w != nullptr) xh = __fmul_rn(xh, qw[k]);
+          q[k] = code_s8(__fmul_rn(xh, sc));
+        }
+        const uint32_t w0 = pack4(q[0], q[1], q[2], q[3]);
+        const uint32_t w1 = pack4(q[4], q[5], q[6], q[7]);
+        rs[u] = __dp4a(static_cast<int>(w1), 0x01010101, __dp4a(static_cast<int>(w0), 0x01010101, 0));
+        if (tb + u < nt) {
+          const int64_t t = t0 + tb + u;
+          *reinterpret_cast<uint2*>(p.A + t * H + 8 * v) = make_uint2(w0, w1);
+          if (threadIdx.x == 0) p.gamma[t] = gm;
+        }
+      }
+      block_reduce<int, false>(rs, red_i, ib, nwarps);
+      if (threadIdx.x == 0 && p.rowsum != nullptr)
+#pragma unroll
+        for (int u = 0; u < kTB; ++u)
+          if (tb + u < nt) p.rowsum[t0 + tb + u] = rs[u];
+    }
+  }
+  if (p.hT != nullptr && t0 + nt == p.T) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) p.hT[8 * v + k] = s[k];
+  }
+}
+
+template <int XDT>
+cudaError_t launch_xdt(const MlgruCall& c, cudaStream_t st) {
+  const int64_t nch = (c.T + kChunk - 1) / kChunk;
+  const float* carry = c.h0;
+  if (nch > 1) {
+    const dim3 ga(static_cast<unsigned>(nch), static_cast<unsigned>((c.H / 8 + kAThreads - 1) / kAThreads));
+    mlgru_chunk_kernel<XDT><<<ga, kAThreads, 0, st>>>(c.I, c.F, c.T, c.H, c.amap, c.bmap);
+    mlgru_carry_kernel<<<static_cast<unsigned>((c.H + 3) / 4), 128, 0, st>>>(
+        c.amap, c.bmap, c.h0, static_cast<int>(nch), c.H, c.carry);
+    carry = c.carry;
+  }
+  OutArgs p;
+  p.I = c.I;
+  p.F = c.F;
+  p.G = c.G;
+  p.T = c.T;
+  p.H = c.H;
+  p.carry = carry;
+  p.norm_w = c.norm_w;
+  p.eps = c.eps;
+  p.o = c.o;
+  p.odt = c.odt;
+  p.q_norm_w = c.q_norm_w;
+  p.q_eps = c.q_eps;
+  p.A = c.A;
+  p.gamma = c.gamma;
+  p.rowsum = c.rowsum;
+  p.hT = c.hT;
+  const unsigned threads = static_cast<unsigned>(c.H / 8);
+  if (c.A != nullptr)
+    mlgru_out_kernel<XDT, true><<<static_cast<unsigned>(nch), threads, 0, st>>>(p);
+  else
+    mlgru_out_kernel<XDT, false><<<static_cast<unsigned>(nch), threads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t mlgru_ws_bytes(int64_t T, int64_t H) {
+  const int64_t nch = (T + kChunk - 1) / kChunk;
+  if (nch <= 1) return 0;
+  const size_t one = (static_cast<size_t>(nch * H) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  return 3 * one;
+}
+
+cudaError_t launch_mlgru(const MlgruCall& c, cudaStream_t s) {
+  return c.xdt == kInF16 ? launch_xdt<kInF16>(c, s) : launch_xdt<kInF32>(c, s);
+}
+
+}  // namespace mmf

@@ -250,6 +250,89 @@ MMF_EXPORT mmf_status mmf_quantize_activations(const void* x, mmf_dtype xdt, int
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
+MMF_EXPORT size_t mmf_mlgru_workspace_bytes(int64_t T, int64_t H) {
+  if (T < 1 || T > kMaxT || H < 256 || H > 4096 || H % 256 != 0) return 0;
+  return mlgru_ws_bytes(T, H);
+}
+
+namespace {
+
+mmf_status mlgru_common(const void* I, const void* F, const void* G, int xdt, int64_t T,
+                        int64_t H, const float* h0, const float* norm_w, float eps, float* hT,
+                        void* ws, size_t ws_bytes, MlgruCall& c) {
+  if (!I || !F || !G) return MMF_ERR_INVALID_ARG;
+  if (check_dtype(xdt) != MMF_OK) return MMF_ERR_INVALID_ARG;
+  if (!(eps > 0.0f) || eps != eps || eps > 1.0f) return MMF_ERR_INVALID_ARG;
+  mmf_status st;
+  if ((st = check_t(T)) != MMF_OK) return st;
+  if (H < 256 || H > 4096 || H % 256 != 0) return MMF_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(I, 16) || !aligned(F, 16) || !aligned(G, 16) || (h0 && !aligned(h0, 16)) ||
+      (norm_w && !aligned(norm_w, 16)) || (hT && !aligned(hT, 16)))
+    return MMF_ERR_ALIGNMENT;
+  const size_t need = mlgru_ws_bytes(T, H);
+  if (need > 0 && (ws == nullptr || ws_bytes < need)) return MMF_ERR_WORKSPACE;
+  if (ws == nullptr && ws_bytes != 0) return MMF_ERR_WORKSPACE;
+  if (ws != nullptr && !aligned(ws, 256)) return MMF_ERR_ALIGNMENT;
+  c = MlgruCall{};
+  c.I = I;
+  c.F = F;
+  c.G = G;
+  c.xdt = xdt == MMF_F16 ? kInF16 : kInF32;
+  c.T = T;
+  c.H = static_cast<int>(H);
+  c.h0 = h0;
+  c.norm_w = norm_w;
+  c.eps = eps;
+  c.hT = hT;
+  if (need > 0) {
+    const size_t one = need / 3;
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    c.amap = reinterpret_cast<float*>(b);
+    c.bmap = reinterpret_cast<float*>(b + one);
+    c.carry = reinterpret_cast<float*>(b + 2 * one);
+  }
+  return MMF_OK;
+}
+
+}  // namespace
+
+MMF_EXPORT mmf_status mmf_mlgru_forward(const void* I, const void* F, const void* G,
+                                        mmf_dtype xdt, int64_t T, int64_t H, const float* h0,
+                                        const float* norm_w, float eps, void* o, mmf_dtype odt,
+                                        float* hT, void* ws, size_t ws_bytes, void* stream) {
+  if (!o || check_dtype(odt) != MMF_OK) return MMF_ERR_INVALID_ARG;
+  MlgruCall c;
+  mmf_status st = mlgru_common(I, F, G, xdt, T, H, h0, norm_w, eps, hT, ws, ws_bytes, c);
+  if (st != MMF_OK) return st;
+  if (!aligned(o, 16)) return MMF_ERR_ALIGNMENT;
+  c.o = o;
+  c.odt = odt == MMF_F16 ? kInF16 : kInF32;
+  return from_cuda(launch_mlgru(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+MMF_EXPORT mmf_status mmf_mlgru_forward_quantized(const void* I, const void* F, const void* G,
+                                                  mmf_dtype xdt, int64_t T, int64_t H,
+                                                  const float* h0, const float* norm_w,
+                                                  float eps, const float* oproj_norm_w,
+                                                  float oproj_eps, int8_t* A, float* gamma,
+                                                  int32_t* rowsum, float* hT, void* ws,
+                                                  size_t ws_bytes, void* stream) {
+  if (!A || !gamma) return MMF_ERR_INVALID_ARG;
+  if (!(oproj_eps > 0.0f) || oproj_eps != oproj_eps || oproj_eps > 1.0f) return MMF_ERR_INVALID_ARG;
+  MlgruCall c;
+  mmf_status st = mlgru_common(I, F, G, xdt, T, H, h0, norm_w, eps, hT, ws, ws_bytes, c);
+  if (st != MMF_OK) return st;
+  if (!aligned(A, 16) || !aligned(gamma, 4) || (rowsum && !aligned(rowsum, 4)) ||
+      (oproj_norm_w && !aligned(oproj_norm_w, 16)))
+    return MMF_ERR_ALIGNMENT;
+  c.q_norm_w = oproj_norm_w;
+  c.q_eps = oproj_eps;
+  c.A = A;
+  c.gamma = gamma;
+  c.rowsum = rowsum;
+  return from_cuda(launch_mlgru(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 MMF_EXPORT mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const float* gamma,
                                                       const int32_t* rowsum, int64_t T, int64_t K,
                                                       const uint8_t* Wp, const float* beta,

@@ -139,3 +139,52 @@ def test_program_init_rejects_on_host():
     bad = (mmf.Projection * 1)(mmf.Projection(A16, 1, None, A16, A16, 200, 256, 0, 0, A16, 1))
     assert L.mmf_program_init(bad, 1, 8, 1e-8, A16, 1 << 30, None) == SHAPE      # K % 128
     assert L.mmf_program_workspace_bytes(bad, 1, 8) == 0
+
+
+# ---------------------------------------------------------------------------------- MLGRU
+def test_mlgru_workspace_sizes():
+    L = mmf.lib()
+    # chunk maps a, b and the carries: three [chunks x H] fp32 arrays, 256-byte rounded
+    assert L.mmf_mlgru_workspace_bytes(32768, 2048) == 3 * 512 * 2048 * 4
+    assert L.mmf_mlgru_workspace_bytes(65, 256) == 3 * 2 * 256 * 4
+    assert L.mmf_mlgru_workspace_bytes(64, 2048) == 0      # one chunk: no scan across chunks
+    assert L.mmf_mlgru_workspace_bytes(1, 4096) == 0
+    assert L.mmf_mlgru_workspace_bytes(100, 200) == 0      # unsupported H
+    assert L.mmf_mlgru_workspace_bytes(0, 256) == 0
+
+
+def mlgru(**kw):
+    a = dict(I=A16, F=A16, G=A16, xdt=1, T=200, H=512, h0=None, w=None, eps=1e-8, o=A16, odt=1,
+             hT=None, ws=A16, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return mmf.lib().mmf_mlgru_forward(a["I"], a["F"], a["G"], a["xdt"], a["T"], a["H"],
+                                       a["h0"], a["w"], a["eps"], a["o"], a["odt"], a["hT"],
+                                       a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(I=None), INVALID), (dict(F=None), INVALID), (dict(G=None), INVALID),
+    (dict(o=None), INVALID), (dict(xdt=3), INVALID), (dict(odt=2), INVALID),
+    (dict(eps=0.0), INVALID), (dict(eps=float("nan")), INVALID), (dict(eps=2.0), INVALID),
+    (dict(T=0), SHAPE), (dict(H=128), SHAPE), (dict(H=768 + 128), SHAPE), (dict(H=4352), SHAPE),
+    (dict(I=A16 + 8), ALIGN), (dict(o=A16 + 2), ALIGN), (dict(h0=A16 + 4), ALIGN),
+    (dict(hT=A16 + 4), ALIGN), (dict(w=A16 + 4), ALIGN), (dict(ws=A16 + 16), ALIGN),
+    (dict(ws=None, wsb=0), WS), (dict(wsb=100), WS), (dict(T=64, ws=None, wsb=8), WS),
+])
+def test_mlgru_rejects_on_host(kw, code):
+    assert mlgru(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(A=None), INVALID), (dict(gamma=None), INVALID), (dict(qeps=0.0), INVALID),
+    (dict(A=A16 + 8), ALIGN), (dict(gamma=A16 + 2), ALIGN), (dict(rowsum=A16 + 2), ALIGN),
+    (dict(qw=A16 + 4), ALIGN), (dict(H=100), SHAPE), (dict(wsb=16), WS),
+])
+def test_mlgru_quantized_rejects_on_host(kw, code):
+    a = dict(I=A16, F=A16, G=A16, xdt=1, T=200, H=512, h0=None, w=None, eps=1e-8, qw=None,
+             qeps=1e-8, A=A16, gamma=A16, rowsum=A16, hT=None, ws=A16, wsb=1 << 20, stream=None)
+    a.update(kw)
+    assert mmf.lib().mmf_mlgru_forward_quantized(
+        a["I"], a["F"], a["G"], a["xdt"], a["T"], a["H"], a["h0"], a["w"], a["eps"], a["qw"],
+        a["qeps"], a["A"], a["gamma"], a["rowsum"], a["hT"], a["ws"], a["wsb"],
+        a["stream"]) == code
