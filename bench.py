@@ -18,6 +18,9 @@ HBM, not L2.
 The headline line times the largest single-GPU workload (the 1.3B-shaped prefill, tensor-bound)
 and, in a "decode" object beside it, the HBM-bound decode workloads (1.3B at 1/8/64 tokens,
 2.7B at 8 tokens), each with its own step time, weight GB/s, roofline fraction and clocks.
+An "mlgru" object times the MLGRU recurrence with its swish gate norm (the step after
+i/f/g_proj), alone and fused with o_proj's activation quantisation, on the 1.3B prefill
+shape, and at one decode token.
 
 Arms:
   default            the CUDA library through its C ABI; the timed region replays CUDA
@@ -75,6 +78,8 @@ def parse_args(argv=None):
                     help="least timed GPU time of each decode entry")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-mlgru", action="store_true",
+                    help="skip the MLGRU recurrence + gate norm entry")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
                     help="target host time of each CPU-baseline leg")
     ap.add_argument("--path", choices=["auto", "program", "launches"], default="auto",
@@ -673,7 +678,100 @@ def run_gpu(args, rank, world, local_rank):
         decode[name]["tokens_per_step"] = dwl.T
         decode[name]["layers_per_step"] = dwl.layers
     head["decode"] = decode
+    if not args.no_mlgru:
+        head["mlgru"] = time_mlgru(args, dev, stream, world, local_rank)
     return head
+
+
+# ----------------------------------------------------------------------------- MLGRU
+# The recurrence and gate norm that follow i/f/g_proj, on the 1.3B prefill shape (T tokens of
+# hidden size H) and at one decode token.
+MLGRU_SHAPE = ("hgrn1p3b_mlgru_t32768", 32768, 2048)
+
+
+def mlgru_bytes(T, H, quantized=False, in_bytes=2):
+    """Algorithmic HBM bytes of one MLGRU call: I, F and G read once and o written once (fp16),
+    or, fused, o_proj's int8 codes, gamma and code sums written instead of o."""
+    out = T * H + 8 * T if quantized else in_bytes * T * H
+    return 3 * in_bytes * T * H + out
+
+
+def time_mlgru(args, dev, stream, world, local_rank):
+    """Times mmf_mlgru_forward and mmf_mlgru_forward_quantized (inputs resident in HBM, larger
+    than L2) and one decode token's call."""
+    import torch
+    import ternary_weight_lm_b200 as mmf
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    name, T, H = MLGRU_SHAPE
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+
+    def rnd(t):
+        return (torch.randn((t, H), generator=gen, device=dev) * 1.5).half()
+
+    I, F, G = rnd(T), rnd(T), rnd(T)
+    o = torch.empty((T, H), dtype=torch.float16, device=dev)
+    A = torch.empty((T, H), dtype=torch.int8, device=dev)
+    gam = torch.empty(T, dtype=torch.float32, device=dev)
+    rs = torch.empty(T, dtype=torch.int32, device=dev)
+    hT = torch.empty(H, dtype=torch.float32, device=dev)
+    ws = mmf.workspace(mmf.mmf_mlgru_workspace_bytes(T, H), dev)
+    I1, F1, G1 = rnd(1), rnd(1), rnd(1)
+    o1 = torch.empty((1, H), dtype=torch.float16, device=dev)
+    h1 = torch.zeros(H, dtype=torch.float32, device=dev)
+
+    def plain():
+        mmf.mmf_mlgru_forward(I, F, G, None, None, 1e-8, o, hT, ws, stream)
+
+    def fused():
+        mmf.mmf_mlgru_forward_quantized(I, F, G, None, None, 1e-8, None, 1e-8, A, gam, rs, hT,
+                                        ws, stream)
+
+    def decode():
+        mmf.mmf_mlgru_forward(I1, F1, G1, h1, None, 1e-8, o1, h1, None, stream)
+
+    hbm = measured_peaks()[0]
+    out = {"workload": name, "T": T, "H": H, "dtype": "f16 in, f16 out (fused: int8 codes out)",
+           "inputs": "seeded N(0, 1.5^2) on the device, 3 x %d MB resident, larger than L2"
+                     % (T * H * 2 // 2 ** 20)}
+    for label, fn, q, n, tokens in (("plain", plain, False, 50, T),
+                                    ("fused_oproj_quant", fused, True, 50, T),
+                                    ("decode_t1", decode, False, 2000, 1)):
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, args.warmup)):
+                fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(gpu_index(local_rank)) as clk:
+            barrier()
+            torch.cuda.synchronize()
+            with torch.cuda.stream(stream):
+                e0.record()
+                for _ in range(n):
+                    fn()
+                e1.record()
+            torch.cuda.synchronize()
+            barrier()
+        ms = reduce_max(e0.elapsed_time(e1) / n, world, dev)
+        assert mmf.mmf_get_device_status() == 0
+        nbytes = mlgru_bytes(tokens, H, q)
+        achieved = nbytes / (ms * 1e-3) / 1e9
+        out[label] = {
+            "ms_per_call": round(ms, 4), "tokens_per_s": round(tokens * world / (ms * 1e-3), 1),
+            "launches_per_call": 1 if tokens <= 64 else 3, "calls": n,
+            "roofline": {"bound": "hbm", "kernel": "mlgru call (chunk maps, carries, outputs)",
+                         "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "bytes_per_call": nbytes,
+                         "peak_source": "measured copy bandwidth"},
+            "clocks": clk.summary()}
+    del I, F, G, o, A, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -890,6 +988,8 @@ def main(argv=None):
                     "gpu_launches": res["launches"],
                     "decode": res["decode"],
                 }
+                if "mlgru" in res:
+                    line["mlgru"] = res["mlgru"]
                 if not args.no_cpu_baseline and world == 1:
                     _, cpu = oracle_tokens_per_s(wl, args.cpu_seconds, dataflow=args.dataflow)
                     line["cpu_baseline"] = cpu

@@ -214,12 +214,12 @@ mmf_status mmf_program_run(void* ws, void* stream);
  *   o_tj = h_tj / sqrt(mean_j h_tj^2 + eps) * w_j * silu(G_tj)
  * with h before the first token = h0 (zero when NULL), in float (exp and reciprocals through
  * the fast intrinsics: relative error a few 1e-6 before the output's own rounding).  Tokens are
- * scanned in chunks of 64; chunk boundaries change only the rounding order of h.
+ * scanned in chunks of 32; chunk boundaries change only the rounding order of h.
  *
  * Shapes: 1 <= T <= 16777216; H a multiple of 256, 256 <= H <= 4096.  I, F, G, o: row-major,
  * 16-byte aligned, all of dtype xdt (I/F/G) and odt (o).  h0, hT, norm_w: [H] fp32 (may be
  * NULL), 16-byte aligned.  ws: mmf_mlgru_workspace_bytes(T, H) bytes, 256-byte aligned (NULL
- * with ws_bytes 0 when that is 0, i.e. T <= 64).  Errors as for the forward; a workspace that
+ * with ws_bytes 0 when that is 0, i.e. T <= 32).  Errors as for the forward; a workspace that
  * is missing or too small: MMF_ERR_WORKSPACE.  Asynchronous on `stream`. */
 size_t mmf_mlgru_workspace_bytes(int64_t T, int64_t H);
 

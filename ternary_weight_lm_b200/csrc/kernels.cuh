@@ -59,7 +59,7 @@ bool prefill_ss_supported(const GemmCall& c);
 cudaError_t launch_prefill_ss(const GemmCall& c, int8_t* w8, cudaStream_t s);
 
 // MLGRU recurrence + swish gate norm over T tokens (chunked scan, three launches; one when
-// T <= 64).  amap/bmap/carry: workspace arrays of [chunks x H] floats (mlgru_ws_bytes).  With A
+// T <= 32).  amap/bmap/carry: workspace arrays of [H x chunks] floats (mlgru_ws_bytes).  With A
 // set, o_proj's codes/gamma/rowsum are written instead of o.
 struct MlgruCall {
   const void* I;

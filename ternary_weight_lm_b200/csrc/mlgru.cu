@@ -13,14 +13,14 @@
 //
 // The recurrence is a chain of affine maps h -> a h + b, which compose associatively, so the T
 // tokens are cut into chunks of kChunk and scanned in three launches:
-//   (A) chunk maps: every (chunk, 8 channels) thread composes its chunk's maps, (a, b);
-//   (B) carries: one warp per channel scans the chunk maps (shuffles over 32 chunks at a time)
-//       into the state entering each chunk;
-//   (C) outputs: one CTA per chunk and all H channels (one 16-byte vector of 8 channels per
-//       thread) runs the chunk from its carry and finishes every token's gate norm with a
-//       block reduction; it writes o in fp16/fp32, or, fused, o_proj's int8 codes, gamma and
-//       code sums computed from o rounded to fp16, the same arithmetic as the activation
-//       pre-pass applied to that fp16 o.
+//   (A) chunk maps: every (chunk, 8 channels) thread composes its chunk's maps, (a, b),
+//       stored channel-major ([H][chunks]) so that (B) reads them coalesced;
+//   (B) carries: one warp per channel scans the chunk maps (shuffles over 32 chunks at a time,
+//       eight rounds of loads in flight) into the state entering each chunk;
+//   (C) outputs: one CTA per chunk and all H channels (4 channels per thread) runs the chunk
+//       from its carry and finishes every token's gate norm with a block reduction; it writes
+//       o in fp16/fp32, or, fused, o_proj's int8 codes, gamma and code sums computed from o
+//       rounded to fp16, the same arithmetic as the activation pre-pass applied to that o.
 // With T <= kChunk, (C) alone runs from the initial state.
 //
 // Rooflines: HBM-bound.  (A) reads I and F, (C) reads I, F and G and writes o: 12 bytes per
@@ -34,7 +34,7 @@
 namespace mmf {
 namespace {
 
-constexpr int kChunk = 64;       // tokens per chunk
+constexpr int kChunk = 32;       // tokens per chunk (1024 chunks, 3.5 waves of (C) at 32768)
 constexpr int kAThreads = 128;   // threads per CTA of the chunk-map kernel
 constexpr int kTB = 4;           // tokens per block reduction in the output kernel
 // |x| cap before exp.  At +-40 a gate is within 5e-18 of its limit, and (1 + e1)(1 + e2) stays
@@ -63,29 +63,43 @@ __device__ __forceinline__ void load8(const void* base, int64_t off, float (&v)[
   }
 }
 
-// One token's map for one channel: h -> f h + (1 - f) c.  With e1 = exp(-F), e2 = exp(-I):
-// f = 1/(1+e1) and sigmoid(I) = 1/(1+e2) come from one reciprocal of (1+e1)(1+e2), and
-// 1 - f = e1 f without cancellation.  Inputs are capped at +-kClamp first.
+// 4 channels of one row as floats: 8 bytes of fp16, or 16 of fp32.
+template <int XDT>
+__device__ __forceinline__ void load4(const void* base, int64_t off, float (&v)[4]) {
+  if (XDT == kInF16) {
+    const uint2 u = *reinterpret_cast<const uint2*>(reinterpret_cast<const __half*>(base) + off);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + off);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  }
+}
+
+// One token's map for one channel: h -> f h + (1 - f) c.  With e1 = exp(-F), e2 = exp(-I) and
+// r = 1 / ((1 + e1)(1 + e2)) (one reciprocal for both gates):
+//   f = 1/(1+e1) = r (1+e2),   (1 - f) silu(I) = e1/(1+e1) * I/(1+e2) = I e1 r,
+// with no cancellation in 1 - f.  Only the upper side of each exponent's argument is capped
+// (kClamp): exp of a large negative argument is 0, which is the limit of the gate.
 __device__ __forceinline__ void token_map(float F, float I, float& f, float& u) {
-  const float e1 = __expf(-fminf(fmaxf(F, -kClamp), kClamp));
-  const float e2 = __expf(-fminf(fmaxf(I, -kClamp), kClamp));
-  const float d1 = 1.0f + e1, d2 = 1.0f + e2;
-  const float r = __fdividef(1.0f, d1 * d2);
+  const float e1 = __expf(fminf(-F, kClamp));
+  const float e2 = __expf(fminf(-I, kClamp));
+  const float d2 = 1.0f + e2;
+  const float r = __fdividef(1.0f, (1.0f + e1) * d2);
   f = r * d2;
-  const float sI = r * d1;
-  u = (e1 * f) * (I * sI);          // (1 - f) * silu(I)
+  u = I * (e1 * r);
 }
 
 __device__ __forceinline__ float silu_f(float g) {
-  const float e = __expf(-fminf(fmaxf(g, -kClamp), kClamp));
-  return g * __fdividef(1.0f, 1.0f + e);
+  return g * __fdividef(1.0f, 1.0f + __expf(fminf(-g, kClamp)));
 }
 
 // ------------------------------------------------------------------------------- (A) chunk maps
 template <int XDT>
 __global__ void __launch_bounds__(kAThreads) mlgru_chunk_kernel(const void* I, const void* F,
-                                                                int64_t T, int H, float* Amap,
-                                                                float* Bmap) {
+                                                                int64_t T, int H, int nch,
+                                                                float* Amap, float* Bmap) {
   const int chunk = blockIdx.x;
   const int v = blockIdx.y * kAThreads + threadIdx.x;    // vector of channels 8v .. 8v+7
   if (8 * v >= H) return;
@@ -129,52 +143,64 @@ __global__ void __launch_bounds__(kAThreads) mlgru_chunk_kernel(const void* I, c
       b[k] = fmaf(f, b[k], w);
     }
   }
-  float4* ao = reinterpret_cast<float4*>(Amap + static_cast<int64_t>(chunk) * H + 8 * v);
-  float4* bo = reinterpret_cast<float4*>(Bmap + static_cast<int64_t>(chunk) * H + 8 * v);
-  ao[0] = make_float4(a[0], a[1], a[2], a[3]);
-  ao[1] = make_float4(a[4], a[5], a[6], a[7]);
-  bo[0] = make_float4(b[0], b[1], b[2], b[3]);
-  bo[1] = make_float4(b[4], b[5], b[6], b[7]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    Amap[static_cast<int64_t>(8 * v + k) * nch + chunk] = a[k];
+    Bmap[static_cast<int64_t>(8 * v + k) * nch + chunk] = b[k];
+  }
 }
 
 // ------------------------------------------------------------------------------- (B) carries
-// One warp per channel.  Lane l takes chunk k0 + l; an inclusive shuffle scan composes the maps
-// of chunks k0 .. k0 + l (later map applied after the earlier one: (a, b) after (a', b') is
+// One warp per channel; maps and carries are channel-major, so lane l reads chunk k0 + l of
+// the channel's contiguous row.  An inclusive shuffle scan composes the maps of chunks
+// k0 .. k0 + l (the later map applied after the earlier one: (a, b) after (a', b') is
 // (a a', a b' + b)); the carry into chunk k is the exclusive composite applied to the state s
-// entering chunk k0.  Lanes past the last chunk hold the identity map.
+// entering chunk k0.  Lanes past the last chunk hold the identity map.  The loads of kRounds
+// rounds are issued before their scans (they do not depend on s).
+constexpr int kRounds = 8;
+
 __global__ void __launch_bounds__(128) mlgru_carry_kernel(const float* Amap, const float* Bmap,
                                                           const float* h0, int nch, int H,
                                                           float* carry) {
   const int j = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (j >= H) return;
+  const float* ar = Amap + static_cast<int64_t>(j) * nch;
+  const float* br = Bmap + static_cast<int64_t>(j) * nch;
+  float* cr = carry + static_cast<int64_t>(j) * nch;
   float s = h0 != nullptr ? h0[j] : 0.0f;
-  for (int k0 = 0; k0 < nch; k0 += 32) {
-    const int k = k0 + lane;
-    float a = 1.0f, b = 0.0f;
-    if (k < nch) {
-      a = Amap[static_cast<int64_t>(k) * H + j];
-      b = Bmap[static_cast<int64_t>(k) * H + j];
+  for (int k0 = 0; k0 < nch; k0 += 32 * kRounds) {
+    float av[kRounds], bv[kRounds];
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+      const int k = k0 + 32 * r + lane;
+      av[r] = k < nch ? ar[k] : 1.0f;
+      bv[r] = k < nch ? br[k] : 0.0f;
     }
 #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const float ap = __shfl_up_sync(0xffffffffu, a, d);
-      const float bp = __shfl_up_sync(0xffffffffu, b, d);
-      if (lane >= d) {
-        b = fmaf(a, bp, b);
-        a *= ap;
+    for (int r = 0; r < kRounds; ++r) {
+      float a = av[r], b = bv[r];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const float ap = __shfl_up_sync(0xffffffffu, a, d);
+        const float bp = __shfl_up_sync(0xffffffffu, b, d);
+        if (lane >= d) {
+          b = fmaf(a, bp, b);
+          a *= ap;
+        }
       }
+      float ae = __shfl_up_sync(0xffffffffu, a, 1);
+      float be = __shfl_up_sync(0xffffffffu, b, 1);
+      if (lane == 0) {
+        ae = 1.0f;
+        be = 0.0f;
+      }
+      const int k = k0 + 32 * r + lane;
+      if (k < nch) cr[k] = fmaf(ae, s, be);
+      const float al = __shfl_sync(0xffffffffu, a, 31);
+      const float bl = __shfl_sync(0xffffffffu, b, 31);
+      s = fmaf(al, s, bl);
     }
-    float ae = __shfl_up_sync(0xffffffffu, a, 1);
-    float be = __shfl_up_sync(0xffffffffu, b, 1);
-    if (lane == 0) {
-      ae = 1.0f;
-      be = 0.0f;
-    }
-    if (k < nch) carry[static_cast<int64_t>(k) * H + j] = fmaf(ae, s, be);
-    const float al = __shfl_sync(0xffffffffu, a, 31);
-    const float bl = __shfl_sync(0xffffffffu, b, 31);
-    s = fmaf(al, s, bl);
   }
 }
 
@@ -197,7 +223,8 @@ struct OutArgs {
   const void* G;
   int64_t T;
   int H;
-  const float* carry;    // [nch x H] state entering each chunk, or (one chunk) h0, or nullptr
+  const float* carry;    // [H x nch] state entering each chunk, or (one chunk) h0, or nullptr
+  int nch;
   const float* norm_w;   // gate norm weight [H] or nullptr
   float eps;
   void* o;               // [T x H] fp16 / fp32 (plain mode)
@@ -241,54 +268,50 @@ __device__ __forceinline__ void block_reduce(V (&x)[kTB], V* red, int& buf, int 
 }
 
 template <int XDT, bool QUANT>
-__global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
+__global__ void __launch_bounds__(1024) mlgru_out_kernel(const OutArgs p) {
   __shared__ float red_f[2 * kTB * 32];
   __shared__ double red_d[2 * kTB * 32];
   __shared__ int red_i[2 * kTB * 32];
   const int chunk = blockIdx.x;
-  const int v = threadIdx.x;                 // channels 8v .. 8v+7
+  const int v = threadIdx.x;                 // channels 4v .. 4v+3
   const int H = p.H;
   const int nwarps = blockDim.x >> 5;
   const int64_t t0 = static_cast<int64_t>(chunk) * kChunk;
   const int nt = static_cast<int>(p.T - t0 < kChunk ? p.T - t0 : kChunk);
-  float s[8], w[8], qw[8];
-  {
-    const float* c = p.carry != nullptr ? p.carry + static_cast<int64_t>(chunk) * H : nullptr;
+  float s[4], w[4], qw[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      s[k] = c != nullptr ? c[8 * v + k] : 0.0f;
-      w[k] = p.norm_w != nullptr ? p.norm_w[8 * v + k] : 1.0f;
-      qw[k] = (QUANT && p.q_norm_w != nullptr) ? p.q_norm_w[8 * v + k] : 1.0f;
-    }
+  for (int k = 0; k < 4; ++k) {
+    const int j = 4 * v + k;
+    s[k] = p.carry == nullptr ? 0.0f
+           : (p.nch > 1 ? p.carry[static_cast<int64_t>(j) * p.nch + chunk] : p.carry[j]);
+    w[k] = p.norm_w != nullptr ? p.norm_w[j] : 1.0f;
+    qw[k] = (QUANT && p.q_norm_w != nullptr) ? p.q_norm_w[j] : 1.0f;
   }
   int fb = 0, db = 0, ib = 0;
   const float invH = 1.0f / static_cast<float>(H);
   for (int tb = 0; tb < nt; tb += kTB) {
-    float hv[kTB][8], gv[kTB][8];
+    float hv[kTB][4], gv[kTB][4];
     float ss[kTB];
+    // the batch's loads first (they do not depend on the state), then the recurrence
+    float iv[kTB][4], fv[kTB][4];
+#pragma unroll
+    for (int u = 0; u < kTB; ++u) {
+      const int64_t off = (t0 + (tb + u < nt ? tb + u : tb)) * H + 4 * v;
+      load4<XDT>(p.I, off, iv[u]);
+      load4<XDT>(p.F, off, fv[u]);
+      load4<XDT>(p.G, off, gv[u]);
+    }
 #pragma unroll
     for (int u = 0; u < kTB; ++u) {
       ss[u] = 0.0f;
-      if (tb + u < nt) {
-        const int64_t off = (t0 + tb + u) * H + 8 * v;
-        float iv[8], fv[8];
-        load8<XDT>(p.I, off, iv);
-        load8<XDT>(p.F, off, fv);
-        load8<XDT>(p.G, off, gv[u]);
+      const bool live = tb + u < nt;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float f, uu;
-          token_map(fv[k], iv[k], f, uu);
-          s[k] = fmaf(f, s[k], uu);
-          hv[u][k] = s[k];
-          ss[u] = fmaf(s[k], s[k], ss[u]);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          hv[u][k] = 0.0f;
-          gv[u][k] = 0.0f;
-        }
+      for (int k = 0; k < 4; ++k) {
+        float f, uu;
+        token_map(fv[u][k], iv[u][k], f, uu);
+        if (live) s[k] = fmaf(f, s[k], uu);
+        hv[u][k] = live ? s[k] : 0.0f;
+        ss[u] = fmaf(hv[u][k], hv[u][k], ss[u]);
       }
     }
     block_reduce<float, false>(ss, red_f, fb, nwarps);
@@ -297,23 +320,23 @@ __global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
     for (int u = 0; u < kTB; ++u) {
       const float inv = __fdiv_rn(1.0f, __fsqrt_rn(fmaf(ss[u], invH, p.eps)));
 #pragma unroll
-      for (int k = 0; k < 8; ++k) hv[u][k] = hv[u][k] * inv * w[k] * silu_f(gv[u][k]);
+      for (int k = 0; k < 4; ++k) hv[u][k] = hv[u][k] * inv * w[k] * silu_f(gv[u][k]);
     }
     if (!QUANT) {
 #pragma unroll
       for (int u = 0; u < kTB; ++u) {
         if (tb + u >= nt) break;
-        const int64_t off = (t0 + tb + u) * H + 8 * v;
+        const int64_t off = (t0 + tb + u) * H + 4 * v;
         if (p.odt == kInF16) {
-          uint4 pk;
-          __half2* h2 = reinterpret_cast<__half2*>(&pk);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) h2[i] = __floats2half2_rn(hv[u][2 * i], hv[u][2 * i + 1]);
-          *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.o) + off) = pk;
+          const __half2 lo = __floats2half2_rn(hv[u][0], hv[u][1]);
+          const __half2 hi = __floats2half2_rn(hv[u][2], hv[u][3]);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+          *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(p.o) + off) = pk;
         } else {
-          float4* d = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + off);
-          d[0] = make_float4(hv[u][0], hv[u][1], hv[u][2], hv[u][3]);
-          d[1] = make_float4(hv[u][4], hv[u][5], hv[u][6], hv[u][7]);
+          *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + off) =
+              make_float4(hv[u][0], hv[u][1], hv[u][2], hv[u][3]);
         }
       }
     } else {
@@ -327,7 +350,7 @@ __global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
         sd[u] = 0.0;
         mx[u] = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
           hv[u][k] = __half2float(__float2half_rn(hv[u][k]));
           const double dx = static_cast<double>(hv[u][k]);
           sd[u] = fma(dx, dx, sd[u]);
@@ -345,7 +368,7 @@ __global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
         } else {
           amax[u] = 0.0f;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+          for (int k = 0; k < 4; ++k)
             amax[u] = fmaxf(amax[u], fabsf(__fmul_rn(__fmul_rn(hv[u][k], inv[u]), qw[k])));
         }
       }
@@ -356,19 +379,18 @@ __global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
         const float gm = fmaxf(p.q_norm_w == nullptr ? __fmul_rn(amax[u], inv[u]) : amax[u],
                                1e-5f);
         const float sc = __fdiv_rn(127.0f, gm);
-        int q[8];
+        int q[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
           float xh = __fmul_rn(hv[u][k], inv[u]);
           if (p.q_norm_w != nullptr) xh = __fmul_rn(xh, qw[k]);
           q[k] = code_s8(__fmul_rn(xh, sc));
         }
         const uint32_t w0 = pack4(q[0], q[1], q[2], q[3]);
-        const uint32_t w1 = pack4(q[4], q[5], q[6], q[7]);
-        rs[u] = __dp4a(static_cast<int>(w1), 0x01010101, __dp4a(static_cast<int>(w0), 0x01010101, 0));
+        rs[u] = __dp4a(static_cast<int>(w0), 0x01010101, 0);
         if (tb + u < nt) {
           const int64_t t = t0 + tb + u;
-          *reinterpret_cast<uint2*>(p.A + t * H + 8 * v) = make_uint2(w0, w1);
+          *reinterpret_cast<uint32_t*>(p.A + t * H + 4 * v) = w0;
           if (threadIdx.x == 0) p.gamma[t] = gm;
         }
       }
@@ -381,7 +403,7 @@ __global__ void __launch_bounds__(512) mlgru_out_kernel(const OutArgs p) {
   }
   if (p.hT != nullptr && t0 + nt == p.T) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) p.hT[8 * v + k] = s[k];
+    for (int k = 0; k < 4; ++k) p.hT[4 * v + k] = s[k];
   }
 }
 
@@ -391,7 +413,8 @@ cudaError_t launch_xdt(const MlgruCall& c, cudaStream_t st) {
   const float* carry = c.h0;
   if (nch > 1) {
     const dim3 ga(static_cast<unsigned>(nch), static_cast<unsigned>((c.H / 8 + kAThreads - 1) / kAThreads));
-    mlgru_chunk_kernel<XDT><<<ga, kAThreads, 0, st>>>(c.I, c.F, c.T, c.H, c.amap, c.bmap);
+    mlgru_chunk_kernel<XDT><<<ga, kAThreads, 0, st>>>(c.I, c.F, c.T, c.H, static_cast<int>(nch),
+                                                      c.amap, c.bmap);
     mlgru_carry_kernel<<<static_cast<unsigned>((c.H + 3) / 4), 128, 0, st>>>(
         c.amap, c.bmap, c.h0, static_cast<int>(nch), c.H, c.carry);
     carry = c.carry;
@@ -403,6 +426,7 @@ cudaError_t launch_xdt(const MlgruCall& c, cudaStream_t st) {
   p.T = c.T;
   p.H = c.H;
   p.carry = carry;
+  p.nch = static_cast<int>(nch);
   p.norm_w = c.norm_w;
   p.eps = c.eps;
   p.o = c.o;
@@ -413,7 +437,7 @@ cudaError_t launch_xdt(const MlgruCall& c, cudaStream_t st) {
   p.gamma = c.gamma;
   p.rowsum = c.rowsum;
   p.hT = c.hT;
-  const unsigned threads = static_cast<unsigned>(c.H / 8);
+  const unsigned threads = static_cast<unsigned>(c.H / 4);
   if (c.A != nullptr)
     mlgru_out_kernel<XDT, true><<<static_cast<unsigned>(nch), threads, 0, st>>>(p);
   else

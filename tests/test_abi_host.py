@@ -145,9 +145,9 @@ def test_program_init_rejects_on_host():
 def test_mlgru_workspace_sizes():
     L = mmf.lib()
     # chunk maps a, b and the carries: three [chunks x H] fp32 arrays, 256-byte rounded
-    assert L.mmf_mlgru_workspace_bytes(32768, 2048) == 3 * 512 * 2048 * 4
-    assert L.mmf_mlgru_workspace_bytes(65, 256) == 3 * 2 * 256 * 4
-    assert L.mmf_mlgru_workspace_bytes(64, 2048) == 0      # one chunk: no scan across chunks
+    assert L.mmf_mlgru_workspace_bytes(32768, 2048) == 3 * 1024 * 2048 * 4
+    assert L.mmf_mlgru_workspace_bytes(65, 256) == 3 * 3 * 256 * 4
+    assert L.mmf_mlgru_workspace_bytes(32, 2048) == 0      # one chunk: no scan across chunks
     assert L.mmf_mlgru_workspace_bytes(1, 4096) == 0
     assert L.mmf_mlgru_workspace_bytes(100, 200) == 0      # unsupported H
     assert L.mmf_mlgru_workspace_bytes(0, 256) == 0
@@ -169,7 +169,7 @@ def mlgru(**kw):
     (dict(T=0), SHAPE), (dict(H=128), SHAPE), (dict(H=768 + 128), SHAPE), (dict(H=4352), SHAPE),
     (dict(I=A16 + 8), ALIGN), (dict(o=A16 + 2), ALIGN), (dict(h0=A16 + 4), ALIGN),
     (dict(hT=A16 + 4), ALIGN), (dict(w=A16 + 4), ALIGN), (dict(ws=A16 + 16), ALIGN),
-    (dict(ws=None, wsb=0), WS), (dict(wsb=100), WS), (dict(T=64, ws=None, wsb=8), WS),
+    (dict(ws=None, wsb=0), WS), (dict(wsb=100), WS), (dict(T=32, ws=None, wsb=8), WS),
 ])
 def test_mlgru_rejects_on_host(kw, code):
     assert mlgru(**kw) == code

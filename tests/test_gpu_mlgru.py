@@ -57,11 +57,11 @@ def _check_state(hT, hT_ref):
     assert np.all(np.abs(hT - hT_ref) <= 1e-4 * (np.abs(hT_ref) + rms))
 
 
-# T around the 64-token chunk (one chunk, a boundary, a ragged second chunk), several chunks,
-# and more than 32 chunks (the carry scan's second round of shuffles); H from one to ten
-# warps of channel vectors.
-@pytest.mark.parametrize("T,H", [(1, 256), (17, 512), (64, 2048), (65, 256), (200, 2560),
-                                 (2577, 1024), (4160, 256)])
+# T around the 32-token chunk (one chunk, a boundary, a ragged second chunk), several chunks,
+# more than 32 chunks (the carry scan's second round of shuffles) and more than 256 (its second
+# batch of prefetched rounds); H from two to twenty warps of channel quads.
+@pytest.mark.parametrize("T,H", [(1, 256), (17, 512), (32, 2048), (33, 256), (200, 2560),
+                                 (2577, 1024), (8230, 256)])
 def test_mlgru_matches_oracle(T, H):
     I, F, G = _inputs(T, H, seed=T + H)
     o, hT = _run(I, F, G)
