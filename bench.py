@@ -138,6 +138,7 @@ KERNEL_SOURCES = {
     "program_kernel": ["program.cu"],
     "ternary_gemm": ["ternary_gemm.cu", "prefill_ss.cu"],
     "act_quant": ["act_quant.cu"],
+    "mlgru": ["mlgru.cu"],
 }
 
 
@@ -767,7 +768,8 @@ def time_mlgru(args, dev, stream, world, local_rank):
             "roofline": {"bound": "hbm", "kernel": "mlgru call (chunk maps, carries, outputs)",
                          "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
                          "frac": round(achieved / hbm, 4), "bytes_per_call": nbytes,
-                         "peak_source": "measured copy bandwidth"},
+                         "peak_source": "measured copy bandwidth",
+                         "traffic": profiled_traffic("mlgru", name) if tokens == T else None},
             "clocks": clk.summary()}
     del I, F, G, o, A, ws
     torch.cuda.empty_cache()
