@@ -91,8 +91,10 @@ __device__ __forceinline__ void token_map(float F, float I, float& f, float& u) 
   u = I * (e1 * r);
 }
 
+// silu(g) = g / (1 + exp(-g)).  No cap: for g below about -88 the exponential is infinite and
+// its reciprocal 0, which is the limit.
 __device__ __forceinline__ float silu_f(float g) {
-  return g * __fdividef(1.0f, 1.0f + __expf(fminf(-g, kClamp)));
+  return g * __fdividef(1.0f, 1.0f + __expf(-g));
 }
 
 // ------------------------------------------------------------------------------- (A) chunk maps
@@ -237,33 +239,46 @@ struct OutArgs {
   float* hT;             // [H] final state or nullptr
 };
 
-// Block reduction of kTB per-thread values of type V (sum or max): every thread gets the
-// totals.  red: 2 buffers x kTB x 32 warps; the buffer alternates, so one barrier per round.
+// Block reduction of the 4 (= kTB) per-thread values of type V (sum, or max of non-negative
+// values): every thread gets the 4 totals.  red: 2 buffers x 4 tokens x 32 warps; the buffer
+// alternates, so one barrier per round.
+//  1. Within a warp a butterfly folds the 4 values as it reduces: after the exchanges at
+//     distance 16 and 8 lane l holds token l/8 only, then distances 4, 2, 1 finish the warp's
+//     sum, and lane 8u stores token u's partial (6 shuffles instead of 20).
+//  2. After the barrier lane l sums token l/8's partials of warps l%8, l%8 + 8, ..., the
+//     eight lanes of a token combine (distances 4, 2, 1), and lanes 0, 8, 16, 24 broadcast the
+//     totals.
+static_assert(kTB == 4, "the reduction folds four tokens");
+
+template <typename V, bool MAX>
+__device__ __forceinline__ V rop(V a, V b) {
+  return MAX ? (b > a ? b : a) : a + b;
+}
+
 template <typename V, bool MAX>
 __device__ __forceinline__ void block_reduce(V (&x)[kTB], V* red, int& buf, int nwarps) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool h16 = (lane & 16) != 0, h8 = (lane & 8) != 0;
+  // keep tokens {0, 1} (lanes 0-15) or {2, 3} (16-31); send the partner the other two
+  V k0 = h16 ? x[2] : x[0], k1 = h16 ? x[3] : x[1];
+  const V s0 = h16 ? x[0] : x[2], s1 = h16 ? x[1] : x[3];
+  k0 = rop<V, MAX>(k0, __shfl_xor_sync(0xffffffffu, s0, 16));
+  k1 = rop<V, MAX>(k1, __shfl_xor_sync(0xffffffffu, s1, 16));
+  V k = h8 ? k1 : k0;
+  const V sd = h8 ? k0 : k1;
+  k = rop<V, MAX>(k, __shfl_xor_sync(0xffffffffu, sd, 8));
 #pragma unroll
-  for (int u = 0; u < kTB; ++u) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const V y = __shfl_xor_sync(0xffffffffu, x[u], o);
-      x[u] = MAX ? (y > x[u] ? y : x[u]) : x[u] + y;
-    }
-  }
+  for (int o = 4; o > 0; o >>= 1) k = rop<V, MAX>(k, __shfl_xor_sync(0xffffffffu, k, o));
   V* r = red + buf * (kTB * 32);
-  if (lane == 0)
-#pragma unroll
-    for (int u = 0; u < kTB; ++u) r[u * 32 + warp] = x[u];
+  const int u = lane >> 3;
+  if ((lane & 7) == 0) r[u * 32 + warp] = k;
   __syncthreads();
+  V acc = V(0);
+  for (int w = lane & 7; w < nwarps; w += 8) acc = rop<V, MAX>(acc, r[u * 32 + w]);
 #pragma unroll
-  for (int u = 0; u < kTB; ++u) {
-    V acc = r[u * 32];
-    for (int w = 1; w < nwarps; ++w) {
-      const V y = r[u * 32 + w];
-      acc = MAX ? (y > acc ? y : acc) : acc + y;
-    }
-    x[u] = acc;
-  }
+  for (int o = 4; o > 0; o >>= 1) acc = rop<V, MAX>(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+#pragma unroll
+  for (int t = 0; t < kTB; ++t) x[t] = __shfl_sync(0xffffffffu, acc, 8 * t);
   buf ^= 1;
 }
 
@@ -301,17 +316,32 @@ __global__ void __launch_bounds__(1024) mlgru_out_kernel(const OutArgs p) {
       load4<XDT>(p.F, off, fv[u]);
       load4<XDT>(p.G, off, gv[u]);
     }
+    if (tb + kTB <= nt) {
 #pragma unroll
-    for (int u = 0; u < kTB; ++u) {
-      ss[u] = 0.0f;
-      const bool live = tb + u < nt;
+      for (int u = 0; u < kTB; ++u) {
+        ss[u] = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float f, uu;
-        token_map(fv[u][k], iv[u][k], f, uu);
-        if (live) s[k] = fmaf(f, s[k], uu);
-        hv[u][k] = live ? s[k] : 0.0f;
-        ss[u] = fmaf(hv[u][k], hv[u][k], ss[u]);
+        for (int k = 0; k < 4; ++k) {
+          float f, uu;
+          token_map(fv[u][k], iv[u][k], f, uu);
+          s[k] = fmaf(f, s[k], uu);
+          hv[u][k] = s[k];
+          ss[u] = fmaf(s[k], s[k], ss[u]);
+        }
+      }
+    } else {   // the last, partial batch of the sequence
+#pragma unroll
+      for (int u = 0; u < kTB; ++u) {
+        ss[u] = 0.0f;
+        const bool live = tb + u < nt;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          float f, uu;
+          token_map(fv[u][k], iv[u][k], f, uu);
+          if (live) s[k] = fmaf(f, s[k], uu);
+          hv[u][k] = live ? s[k] : 0.0f;
+          ss[u] = fmaf(hv[u][k], hv[u][k], ss[u]);
+        }
       }
     }
     block_reduce<float, false>(ss, red_f, fb, nwarps);
