@@ -41,6 +41,7 @@ def _L():
         D = ctypes.c_double
         lib.orc_mlgru_scan.argtypes = [P, P, I64, I64, P, P, P]
         lib.orc_swish_gate_norm.argtypes = [P, P, I64, I64, P, D, P]
+        lib.orc_bitlinear_backward.argtypes = [P, I64, I64, P, D, P, P, P, F, I64, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -207,3 +208,29 @@ def mlgru_forward(I, F, G, h0=None, w=None, eps=1e-8):
     """Recurrence then the swish gate norm.  Returns ``(o [T, H] double, hT [H] double)``."""
     h, hT = mlgru_scan(I, F, h0)
     return swish_gate_norm(h, G, w, eps), hT
+
+
+def bitlinear_backward(x, q, gamma, c, beta, dy, g=None, eps=1e-8, want_dg=True):
+    """Straight-through backward of the projection, in double.
+
+    ``x`` [T, K] (the forward input), ``q`` [T, K] int8 and ``gamma`` [T] (the forward's
+    activation codes and scales), ``c`` [N, K] int8 and ``beta`` (the weight codes and scale),
+    ``dy`` [T, N].  Returns ``(dx [T, K], dW [N, K], dg [K] or None)``.
+    """
+    x = _f64(x)
+    dy = _f64(dy)
+    T, K = x.shape
+    N = dy.shape[1]
+    assert dy.shape[0] == T
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    c = np.ascontiguousarray(c, dtype=np.int8)
+    assert q.shape == (T, K) and c.shape == (N, K)
+    gamma = _f32(gamma)
+    gg = None if g is None else _f64(g)
+    dx = np.empty((T, K), dtype=np.float64)
+    dW = np.empty((N, K), dtype=np.float64)
+    dg = np.empty(K, dtype=np.float64) if want_dg else None
+    _L().orc_bitlinear_backward(_p(x), T, K, None if gg is None else _p(gg), float(eps), _p(q),
+                                _p(gamma), _p(c), float(np.float32(beta)), N, _p(dy), _p(dx),
+                                _p(dW), None if dg is None else _p(dg))
+    return dx, dW, dg

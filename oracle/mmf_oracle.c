@@ -43,6 +43,9 @@
  *    given (zero by default); all in double.
  *  - FusedRMSNormSwishGate: o = (h / sqrt(mean_j h_j^2 + eps)) * w * silu(g_proj output), the
  *    mean over the H channels of one token, in double.
+ *  - backward (the pages give none): straight-through through both quantisers, i.e. the
+ *    gradient of the bilinear map of the dequantised operands, then of the RMSNorm; the latent
+ *    weight takes the quantised weight's gradient; in double.
  *
  * Every decision that turns a float into an integer (an activation code, a weight code) is made
  * in IEEE single precision, the precision the GPU path uses for the same decision.
@@ -337,4 +340,60 @@ ORC_API void orc_swish_gate_norm(const double* h, const double* G, int64_t T, in
       o[t * H + j] = hr[j] / r * (w ? w[j] : 1.0) * sg;
     }
   }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* FusedBitLinear backward.  The pages print no backward pass.  [P4] "MatMul durch ternäre      */
+/* Operationen ersetzen" says the weights are trained in full precision and mapped to ternary   */
+/* values by absmean quantisation during training: the quantisers sit inside the training       */
+/* forward pass.  Reading taken (straight-through): rounding and clamping in both quantisers    */
+/* pass the gradient unchanged, so the layer is differentiated as the bilinear map of its       */
+/* dequantised operands after the RMSNorm,                                                      */
+/*     y_tn  = sum_k xq_tk * wq_nk,   xq_tk = q_tk * gamma_t / 127,   wq_nk = c_nk * beta,      */
+/*     xhat_tk = x_tk / r_t * g_k,    r_t = sqrt(mean_k x_tk^2 + eps),                          */
+/* where the latent full-precision weight receives the gradient of wq and the quantiser's input */
+/* xhat receives the gradient of xq.  In reverse order of the forward pass:                     */
+/*     dW_nk  = sum_t dy_tn * xq_tk                                                              */
+/*     dxh_tk = sum_n dy_tn * wq_nk                                                              */
+/*     dx_tk  = g_k * dxh_tk / r_t - x_tk / (K r_t^3) * sum_j g_j * dxh_tj * x_tj               */
+/*     dg_k   = sum_t dxh_tk * x_tk / r_t                                                        */
+/* x: [T x K]; g: [K] or NULL (all ones); q [T x K] and gamma [T]: the forward pass's codes and */
+/* scales; c: [N x K] weight codes, beta their scale; dy: [T x N], the gradient of y.  Outputs: */
+/* dx [T x K], dW [N x K], dg [K] (skipped when NULL).  Double throughout.                      */
+ORC_API void orc_bitlinear_backward(const double* x, int64_t T, int64_t K, const double* g,
+                                    double eps, const int8_t* q, const float* gamma,
+                                    const int8_t* c, float beta, int64_t N, const double* dy,
+                                    double* dx, double* dW, double* dg) {
+  double* dxh = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int64_t i = 0; i < N * K; ++i) dW[i] = 0.0;
+  if (dg)
+    for (int64_t k = 0; k < K; ++k) dg[k] = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    const double a = (double)gamma[t] / 127.0;
+    /* weights: every output n of this token adds dy_tn times the token's dequantised codes */
+    for (int64_t n = 0; n < N; ++n) {
+      const double d = dy[t * N + n];
+      for (int64_t k = 0; k < K; ++k) dW[n * K + k] += d * ((double)q[t * K + k] * a);
+    }
+    /* through the activation quantiser: the gradient of the dequantised codes */
+    for (int64_t k = 0; k < K; ++k) {
+      double s = 0.0;
+      for (int64_t n = 0; n < N; ++n) s += dy[t * N + n] * ((double)c[n * K + k] * (double)beta);
+      dxh[k] = s;
+    }
+    /* through the RMSNorm */
+    double ss = 0.0, dot = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+      const double xv = x[t * K + k];
+      ss += xv * xv;
+      dot += (g ? g[k] : 1.0) * dxh[k] * xv;
+    }
+    const double r = sqrt(ss / (double)K + eps);
+    for (int64_t k = 0; k < K; ++k) {
+      const double xv = x[t * K + k];
+      dx[t * K + k] = (g ? g[k] : 1.0) * dxh[k] / r - xv * dot / ((double)K * r * r * r);
+      if (dg) dg[k] += dxh[k] * xv / r;
+    }
+  }
+  free(dxh);
 }

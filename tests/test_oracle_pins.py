@@ -405,3 +405,103 @@ def test_swish_gate_norm_scale_invariance_and_zero_gate():
     om = oracle.swish_gate_norm(h, -G, None, 1e-8)
     r = np.sqrt((h * h).mean(axis=1) + 1e-8)[:, None]
     np.testing.assert_allclose((op - om) * r / h, G, rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------------------------
+# Straight-through backward.  The pins differentiate, by central differences in double, the
+# continuous function the straight-through reading differentiates: the RMSNorm followed by the
+# bilinear map of dequantised operands, with the codes held fixed.  The loss is L = sum(dy * y),
+# so a difference quotient of L is one entry of the gradient; none of it calls the backward.
+
+def _surrogate_parts(T, K, N, seed, with_g=True):
+    x = _rand((T, K), seed)
+    g = (0.5 + np.abs(_rand((K,), seed + 1))) if with_g else None
+    W = _rand((N, K), seed + 2)
+    beta = oracle.absmean_beta(W)
+    c = oracle.ternary_codes(W, beta)
+    q, gamma, _ = oracle.rmsnorm_actquant(x.astype(np.float32), g, 1e-8)
+    dy = _rand((T, N), seed + 3)
+    return x, g, q, gamma, c, beta, dy
+
+
+def _norm(x, g, eps):
+    r = np.sqrt((x * x).mean(axis=1, keepdims=True) + eps)
+    return x / r * (1.0 if g is None else g)
+
+
+def test_backward_dx_is_the_gradient_of_norm_then_projection():
+    # L(x) = sum dy * (norm(x) @ (beta c)^T): the surrogate's input gradient, entry by entry
+    T, K, N, eps = 3, 48, 20, 1e-3
+    x, g, q, gamma, c, beta, dy = _surrogate_parts(T, K, N, 41)
+    dx, _, _ = oracle.bitlinear_backward(x, q, gamma, c, beta, dy, g=g, eps=eps)
+    wq = c.astype(np.float64) * float(beta)
+
+    def L(xx):
+        return float((dy * (_norm(xx, g, eps) @ wq.T)).sum())
+    h = 1e-6
+    for t in range(T):
+        for k in (0, 7, 19, 47):
+            e = np.zeros_like(x)
+            e[t, k] = h
+            fd = (L(x + e) - L(x - e)) / (2 * h)
+            assert abs(dx[t, k] - fd) <= 1e-7 * (1 + abs(fd)), (t, k, dx[t, k], fd)
+
+
+def test_backward_dw_is_the_gradient_of_the_dequantised_product():
+    # L(wq) = sum dy * ((q gamma / 127) @ wq^T) with the activation codes held fixed
+    T, K, N = 5, 32, 12
+    x, g, q, gamma, c, beta, dy = _surrogate_parts(T, K, N, 43)
+    _, dW, _ = oracle.bitlinear_backward(x, q, gamma, c, beta, dy, g=g)
+    xq = q.astype(np.float64) * (gamma.astype(np.float64) / 127.0)[:, None]
+    wq = c.astype(np.float64) * float(beta)
+
+    def L(w):
+        return float((dy * (xq @ w.T)).sum())
+    h = 1e-3   # L is linear in w: the quotient is exact up to rounding
+    for n, k in [(0, 0), (3, 31), (11, 5), (7, 16)]:
+        e = np.zeros_like(wq)
+        e[n, k] = h
+        fd = (L(wq + e) - L(wq - e)) / (2 * h)
+        assert abs(dW[n, k] - fd) <= 1e-9 * (1 + abs(fd)), (n, k, dW[n, k], fd)
+
+
+def test_backward_dg_is_the_gradient_of_the_norm_weight():
+    T, K, N, eps = 4, 40, 9, 1e-8
+    x, g, q, gamma, c, beta, dy = _surrogate_parts(T, K, N, 47)
+    _, _, dg = oracle.bitlinear_backward(x, q, gamma, c, beta, dy, g=g, eps=eps)
+    wq = c.astype(np.float64) * float(beta)
+
+    def L(gg):
+        return float((dy * (_norm(x, gg, eps) @ wq.T)).sum())
+    h = 1e-6
+    for k in (0, 13, 39):
+        e = np.zeros_like(g)
+        e[k] = h
+        fd = (L(g + e) - L(g - e)) / (2 * h)
+        assert abs(dg[k] - fd) <= 1e-7 * (1 + abs(fd)), (k, dg[k], fd)
+
+
+def test_backward_input_gradient_is_orthogonal_to_the_input_without_eps():
+    # with eps = 0 the norm is invariant to scaling x, so sum_k x_tk dx_tk = 0 for every token
+    T, K, N = 6, 64, 24
+    x, g, q, gamma, c, beta, dy = _surrogate_parts(T, K, N, 53)
+    dx, _, _ = oracle.bitlinear_backward(x, q, gamma, c, beta, dy, g=g, eps=0.0)
+    dots = (x * dx).sum(axis=1)
+    assert np.all(np.abs(dots) <= 1e-12 * np.abs(x).sum(axis=1) * np.abs(dx).sum(axis=1))
+    # and with eps > 0 it is not (the pin above would catch a dropped eps)
+    dx2, _, _ = oracle.bitlinear_backward(x, q, gamma, c, beta, dy, g=g, eps=1.0)
+    assert np.abs((x * dx2).sum(axis=1)).max() > 1e-3
+
+
+def test_backward_identity_norm_and_unit_codes():
+    # K = 1, g = 1, eps -> 0: xhat = sign(x), so dx = 0; dW_n = dy_n * q * gamma / 127
+    x = np.array([[2.5], [-0.75]])
+    q = np.array([[127], [-127]], dtype=np.int8)
+    gamma = np.array([1.0, 1.0], dtype=np.float32)
+    c = np.array([[1], [-1], [0]], dtype=np.int8)
+    dy = np.array([[1.0, 2.0, 3.0], [-1.0, 0.5, 4.0]])
+    dx, dW, dg = oracle.bitlinear_backward(x, q, gamma, c, 0.5, dy, eps=0.0)
+    assert np.all(np.abs(dx) < 1e-15)
+    np.testing.assert_allclose(dW[:, 0], [1.0 * 1 + (-1.0) * -1, 2.0 - 0.5, 3.0 - 4.0], rtol=1e-15)
+    # dxh_t = sum_n dy_tn c_n beta = (dy_t0 - dy_t1) * 0.5; dg = sum_t dxh_t * x_t / |x_t|
+    np.testing.assert_allclose(dg, [(1.0 - 2.0) * 0.5 * 1 + (-1.0 - 0.5) * 0.5 * -1], rtol=1e-15)
