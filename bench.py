@@ -60,6 +60,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_INT8_TOPS = 4500.0          # B200 dense int8, datasheet
 INT8_PER_BF16 = 2.0                 # nominal dense int8 / bf16 throughput ratio
 GRAPH_SAMPLES = 8                   # distinct step graphs carrying per-launch timing events
+# The straight-through backward leg: one 1.3B layer's six projections (hidden 2048, MLP 5632)
+# at the prefill length: i/f/g/o 2048 -> 2048, gate 2048 -> 11264 (the GLU's 2I rows), down
+# 5632 -> 2048.
+BACKWARD_SHAPE = ("hgrn1p3b_layer_backward_t32768", 32768, 2048, 5632)
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -78,6 +82,10 @@ def parse_args(argv=None):
                     help="least timed GPU time of each decode entry")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the straight-through backward leg")
+    ap.add_argument("--backward-tokens", type=int, default=BACKWARD_SHAPE[1],
+                    help="tokens of the backward leg (smaller for a profiler capture)")
     ap.add_argument("--no-mlgru", action="store_true",
                     help="skip the MLGRU recurrence + gate norm entry")
     ap.add_argument("--cpu-seconds", type=float, default=8.0,
@@ -136,16 +144,17 @@ def tensor_peak(clocks, bf16_burst, bf16_sustained):
 # the sources each profiled kernel is built from (its own file plus the shared device headers)
 KERNEL_SOURCES = {
     "program_kernel": ["program.cu"],
-    "ternary_gemm": ["ternary_gemm.cu", "prefill_ss.cu"],
+    "ternary_gemm": ["ternary_gemm.cu", "prefill_ss.cu", "backward.cuh"],
     "act_quant": ["act_quant.cu"],
     "mlgru": ["mlgru.cu"],
+    "backward": ["backward.cu", "backward.cuh", "prefill_ss.cu"],
 }
 
 
 def kernel_source_sha(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "ternary_weight_lm_b200", "csrc")
-    for name in sorted(KERNEL_SOURCES[kernel] + ["kernels.cuh", "ptx.cuh"]):
+    for name in sorted(set(KERNEL_SOURCES[kernel] + ["kernels.cuh", "ptx.cuh"])):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -681,6 +690,8 @@ def run_gpu(args, rank, world, local_rank):
     head["decode"] = decode
     if not args.no_mlgru:
         head["mlgru"] = time_mlgru(args, dev, stream, world, local_rank)
+    if not args.no_backward:
+        head["backward"] = time_backward(args, dev, stream, world, local_rank)
     return head
 
 
@@ -772,6 +783,123 @@ def time_mlgru(args, dev, stream, world, local_rank):
                          "traffic": profiled_traffic("mlgru", name) if tokens == T else None},
             "clocks": clk.summary()}
     del I, F, G, o, A, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------- backward
+def time_backward(args, dev, stream, world, local_rank):
+    """Times, per projection, the input-gradient call (dx: codes transposed, fp16 contraction
+    over N, norm step) and the weight-gradient call (dW: gradient and codes transposed, fp16
+    contraction over the tokens), with the forward's inputs, codes and the output gradients
+    resident in HBM.  Events between the calls split a step into its two halves."""
+    import torch
+    import ternary_weight_lm_b200 as mmf
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    name, T, H, I = BACKWARD_SHAPE
+    if args.backward_tokens != T:
+        T = args.backward_tokens
+        name = f"hgrn1p3b_layer_backward_t{T}"
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    projs = [("i", "attn", H, H), ("f", "attn", H, H), ("g", "attn", H, H), ("o", "o", H, H),
+             ("gate", "mlp", H, 2 * I), ("down", "h", I, H)]
+    xs, codes = {}, {}
+    for src, K in (("attn", H), ("o", H), ("mlp", H), ("h", I)):
+        x = torch.randn((T, K), generator=gen, device=dev).half()
+        A = torch.empty((T, K), dtype=torch.int8, device=dev)
+        gam = torch.empty(T, dtype=torch.float32, device=dev)
+        torch.cuda.synchronize()     # x was written on the current stream
+        mmf.mmf_quantize_activations(x, None, 1e-8, A, gam, None, stream)
+        xs[src], codes[src] = x, (A, gam)
+    ps = []
+    for pname, src, K, N in projs:
+        W = torch.randn((N, K), generator=gen, device=dev) * 0.02
+        Wp, beta = mmf.quantize_weights(W, stream)
+        torch.cuda.synchronize()
+        del W
+        dy = torch.randn((T, N), generator=gen, device=dev).half()
+        dx = torch.empty((T, K), dtype=torch.float16, device=dev)
+        dW = torch.empty((N, K), dtype=torch.float32, device=dev)
+        ps.append((pname, src, K, N, Wp, beta, dy, dx, dW))
+    ws = mmf.workspace(max(mmf.mmf_backward_workspace_bytes(T, K, N) for _, _, K, N in projs),
+                       dev)
+    torch.cuda.synchronize()
+
+    def step(marks=None):
+        for pname, src, K, N, Wp, beta, dy, dx, dW in ps:
+            A, gam = codes[src]
+            mmf.mmf_bitlinear_backward(xs[src], None, 1e-8, A, gam, Wp, beta, N, dy, dx, None,
+                                       None, ws, stream)
+            if marks is not None:
+                marks.append(("dgrad", 2.0 * T * N * K, torch.cuda.Event(enable_timing=True)))
+                marks[-1][2].record(stream)
+            mmf.mmf_bitlinear_backward(xs[src], None, 1e-8, A, gam, Wp, beta, N, dy, None, dW,
+                                       None, ws, stream)
+            if marks is not None:
+                marks.append(("wgrad", 2.0 * T * N * K, torch.cuda.Event(enable_timing=True)))
+                marks[-1][2].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    torch.cuda.synchronize()
+    n = 8
+    marks = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_index(local_rank)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record()
+            for _ in range(n):
+                step(marks)
+            e1.record()
+        torch.cuda.synchronize()
+        barrier()
+    ms = reduce_max(e0.elapsed_time(e1) / n, world, dev)
+    if mmf.mmf_get_device_status() != 0:
+        raise RuntimeError("device status reported a timeout in the backward leg")
+    # each call's time runs from the previous mark (the timed region's start for the first)
+    halves = {"dgrad": [0.0, 0.0], "wgrad": [0.0, 0.0]}
+    prev = e0
+    for kind, flops, ev in marks:
+        halves[kind][0] += prev.elapsed_time(ev)
+        halves[kind][1] += flops
+        prev = ev
+    flops_step = sum(4.0 * T * N * K for _, _, K, N, *_ in ps)
+    _, bf16_burst, bf16_sust, peak_kind = measured_peaks()
+    step_tflops = flops_step / (ms * 1e-3) / 1e12
+    out = {"workload": name, "T": T, "hidden": H, "mlp": I,
+           "projections": {p[0]: {"K": p[2], "N": p[3]} for p in ps},
+           "dtype": "fp16 operands, fp32 accumulators (dx fp16, dW fp32)",
+           "inputs": "seeded N(0,1) inputs and output gradients and the forward's codes, "
+                     "resident in HBM",
+           "ms_per_step": round(ms, 4), "tokens_per_s": round(T * world / (ms * 1e-3), 1),
+           "steps": n, "calls_per_step": 2 * len(ps), "step_tflops": round(step_tflops, 1),
+           "roofline": {"bound": "tensor", "kernel": "whole backward step",
+                        "achieved": round(step_tflops, 1), "peak": round(bf16_burst, 1),
+                        "unit": "TFLOP/s", "frac": round(step_tflops / bf16_burst, 4),
+                        "peak_source": f"{peak_kind} bf16 dense burst (fp16 runs at the same "
+                                       f"nominal rate)"},
+           "clocks": clk.summary()}
+    for kind, (t_ms, fl) in halves.items():
+        achieved = fl / (t_ms * 1e-3) / 1e12
+        out[kind] = {
+            "ms_per_step": round(t_ms / n, 4),
+            "roofline": {"bound": "tensor",
+                         "kernel": kind + " calls: the fp16 pair GEMM (kind::f16) with the "
+                                          "transpose and norm launches around it",
+                         "achieved": round(achieved, 1), "peak": round(bf16_burst, 1),
+                         "unit": "TFLOP/s", "frac": round(achieved / bf16_burst, 4),
+                         "frac_of_sustained": round(achieved / bf16_sust, 4),
+                         "flops_per_step": fl / n}}
+    del ps, xs, codes, ws
     torch.cuda.empty_cache()
     return out
 
@@ -990,8 +1118,9 @@ def main(argv=None):
                     "gpu_launches": res["launches"],
                     "decode": res["decode"],
                 }
-                if "mlgru" in res:
-                    line["mlgru"] = res["mlgru"]
+                for k in ("mlgru", "backward"):
+                    if k in res:
+                        line[k] = res[k]
                 if not args.no_cpu_baseline and world == 1:
                     _, cpu = oracle_tokens_per_s(wl, args.cpu_seconds, dataflow=args.dataflow)
                     line["cpu_baseline"] = cpu

@@ -241,6 +241,37 @@ mmf_status mmf_mlgru_forward_quantized(const void* I, const void* F, const void*
                                        float* gamma, int32_t* rowsum, float* hT, void* ws,
                                        size_t ws_bytes, void* stream);
 
+/* ---- backward (straight-through) ------------------------------------------------------------
+ * The pages print no backward pass.  [P4] "MatMul durch ternäre Operationen ersetzen": the
+ * weights are trained in full precision and quantised to {-1,0,1} during training, i.e. both
+ * quantisers sit inside the training forward pass.  The library takes the straight-through
+ * reading: rounding and clamping pass the gradient unchanged, so the gradient is that of the
+ * bilinear map of the dequantised operands (xq_tk = q_tk * gamma_t/127, wq_nk = c_nk * beta)
+ * after the RMSNorm (xhat = x / r * g, r as in the forward), with the latent weight taking
+ * wq's gradient.  For the loss gradient dy [T x N] of the forward's y:
+ *   dW_nk  = sum_t dy_tn * xq_tk                                        (fp32 [N x K])
+ *   dxh_tk = beta * sum_n dy_tn * c_nk
+ *   dx_tk  = g_k dxh_tk / r_t - x_tk (sum_j g_j dxh_tj x_tj) / (K r_t^3)   (dxdt [T x K])
+ *   dg_k   = sum_t dxh_tk * x_tk / r_t                                  (fp32 [K])
+ * Both sums over n and t run on the tensor cores with fp16 operands and fp32 accumulation:
+ * dy and the codes are exact in fp16, dy_tn * gamma_t/127 is rounded once to fp16 (relative
+ * error at most 2^-11 per term of dW).  r_t and the norm step are float.
+ *
+ * x, xdt, T, K, norm_w, eps, Wp, beta, N: as passed to the forward.  A [T x K] int8 and gamma
+ * [T]: the forward's activation codes and scales (from mmf_quantize_activations), or both NULL
+ * to have the call recompute them from x.  dy: fp16 [T x N], row-major.  dx (dxdt f32 or f16),
+ * dW and dnorm_w: outputs, each may be NULL to skip it (at least one must be given); they are
+ * overwritten, not accumulated into.  ws: mmf_backward_workspace_bytes(T, K, N) bytes, 256-byte
+ * aligned.  Errors as for the forward.  Asynchronous on `stream` (up to nine launches). */
+size_t mmf_backward_workspace_bytes(int64_t T, int64_t K, int64_t N);
+
+mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
+                                  const float* norm_w, float eps, const int8_t* A,
+                                  const float* gamma, const uint8_t* Wp, const float* beta,
+                                  int64_t N, const void* dy, void* dx, mmf_dtype dxdt,
+                                  float* dW, float* dnorm_w, void* ws, size_t ws_bytes,
+                                  void* stream);
+
 /* ---- forward without any allocation ------------------------------------------------------ */
 
 /* The pages have no counterpart to this entry point; it serves callers that cannot call

@@ -375,11 +375,12 @@ ORC_API void orc_bitlinear_backward(const double* x, int64_t T, int64_t K, const
       const double d = dy[t * N + n];
       for (int64_t k = 0; k < K; ++k) dW[n * K + k] += d * ((double)q[t * K + k] * a);
     }
-    /* through the activation quantiser: the gradient of the dequantised codes */
-    for (int64_t k = 0; k < K; ++k) {
-      double s = 0.0;
-      for (int64_t n = 0; n < N; ++n) s += dy[t * N + n] * ((double)c[n * K + k] * (double)beta);
-      dxh[k] = s;
+    /* through the activation quantiser: the gradient of the dequantised codes (each dxh[k]
+       sums its terms in ascending n; the loops run n-outer only to read c row by row) */
+    for (int64_t k = 0; k < K; ++k) dxh[k] = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      const double d = dy[t * N + n];
+      for (int64_t k = 0; k < K; ++k) dxh[k] += d * ((double)c[n * K + k] * (double)beta);
     }
     /* through the RMSNorm */
     double ss = 0.0, dot = 0.0;

@@ -79,6 +79,9 @@ def lib():
                                                 I),
             "mmf_ternary_accumulate_i32": ([P, I64, I64, P, I64, P, P, SZ, P], I),
             "mmf_bitlinear_forward_noalloc": ([P, I, I64, I64, P, F, P, P, I64, P, I, P], I),
+            "mmf_backward_workspace_bytes": ([I64, I64, I64], SZ),
+            "mmf_bitlinear_backward": ([P, I, I64, I64, P, F, P, P, P, P, I64, P, P, I, P, P, P,
+                                        SZ, P], I),
             "mmf_mlgru_workspace_bytes": ([I64, I64], SZ),
             "mmf_mlgru_forward": ([P, P, P, I, I64, I64, P, P, F, P, I, P, P, SZ, P], I),
             "mmf_mlgru_forward_quantized": ([P, P, P, I, I64, I64, P, P, F, P, F, P, P, P, P, P,
@@ -204,6 +207,21 @@ def mmf_bitlinear_forward_noalloc(x, norm_w, eps, Wp, beta, N, y, stream=None):
     _check("mmf_bitlinear_forward_noalloc", lib().mmf_bitlinear_forward_noalloc(
         _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(Wp), _ptr(beta), N, _ptr(y),
         _dt(y), _stream(stream)))
+
+
+def mmf_backward_workspace_bytes(T, K, N):
+    return lib().mmf_backward_workspace_bytes(T, K, N)
+
+
+def mmf_bitlinear_backward(x, norm_w, eps, A, gamma, Wp, beta, N, dy, dx, dW, dnorm_w, ws,
+                           stream=None):
+    """Straight-through backward (include/mmf.h).  A/gamma: the forward's codes and scales or
+    both None; dx, dW, dnorm_w: outputs or None (dx's dtype selects dxdt)."""
+    T, K = x.shape
+    _check("mmf_bitlinear_backward", lib().mmf_bitlinear_backward(
+        _ptr(x), _dt(x), T, K, _ptr(norm_w), float(eps), _ptr(A), _ptr(gamma), _ptr(Wp),
+        _ptr(beta), N, _ptr(dy), _ptr(dx), MMF_F32 if dx is None else _dt(dx), _ptr(dW),
+        _ptr(dnorm_w), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def mmf_mlgru_workspace_bytes(T, H):
@@ -348,3 +366,21 @@ def bitlinear_glu_forward(x, Wp, beta, norm_w=None, eps=1e-8, out_dtype=None, ws
         ws = workspace(mmf_forward_workspace_bytes(T, K, N2), x.device)
     mmf_bitlinear_glu_forward(x, norm_w, eps, Wp, beta, N2, h, ws, stream)
     return h
+
+
+def bitlinear_backward(x, Wp, beta, dy, norm_w=None, eps=1e-8, A=None, gamma=None,
+                       dx_dtype=None, want_dx=True, want_dW=True, want_dnorm_w=False, ws=None,
+                       stream=None):
+    """Straight-through backward of bitlinear_forward: returns ``(dx, dW, dnorm_w)`` (None for
+    what was not asked).  dy: fp16 [T, N]; dW and dnorm_w are fp32."""
+    import torch
+    T, K = x.shape
+    N = Wp.shape[0]
+    dev = x.device
+    dx = torch.empty((T, K), dtype=dx_dtype or x.dtype, device=dev) if want_dx else None
+    dW = torch.empty((N, K), dtype=torch.float32, device=dev) if want_dW else None
+    dg = torch.empty(K, dtype=torch.float32, device=dev) if want_dnorm_w else None
+    if ws is None:
+        ws = workspace(mmf_backward_workspace_bytes(T, K, N), dev)
+    mmf_bitlinear_backward(x, norm_w, eps, A, gamma, Wp, beta, N, dy, dx, dW, dg, ws, stream)
+    return dx, dW, dg

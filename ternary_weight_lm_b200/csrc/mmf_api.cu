@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/mmf.h"
+#include "backward.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -368,6 +369,57 @@ MMF_EXPORT mmf_status mmf_bitlinear_forward_quantized(const int8_t* A, const flo
   c.wait_limit_ns = kWaitLimitNs;
   c.w8 = (ws != nullptr && w8_ws_bytes(T, K, N) > 0) ? reinterpret_cast<int8_t*>(ws) : nullptr;
   return from_cuda(launch_ternary_gemm(c, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+MMF_EXPORT size_t mmf_backward_workspace_bytes(int64_t T, int64_t K, int64_t N) {
+  if (check_t(T) != MMF_OK || check_k(K) != MMF_OK || check_n(N) != MMF_OK) return 0;
+  return bwd_ws_bytes(T, K, N);
+}
+
+MMF_EXPORT mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
+                                             const float* norm_w, float eps, const int8_t* A,
+                                             const float* gamma, const uint8_t* Wp,
+                                             const float* beta, int64_t N, const void* dy,
+                                             void* dx, mmf_dtype dxdt, float* dW,
+                                             float* dnorm_w, void* ws, size_t ws_bytes,
+                                             void* stream) {
+  if (!x || !Wp || !beta || !dy) return MMF_ERR_INVALID_ARG;
+  if (!dx && !dW && !dnorm_w) return MMF_ERR_INVALID_ARG;
+  if ((A == nullptr) != (gamma == nullptr)) return MMF_ERR_INVALID_ARG;
+  if (check_dtype(xdt) != MMF_OK || check_dtype(dxdt) != MMF_OK) return MMF_ERR_INVALID_ARG;
+  if (!(eps > 0.0f) || eps != eps || eps > 1.0f) return MMF_ERR_INVALID_ARG;
+  mmf_status st;
+  if ((st = check_t(T)) != MMF_OK || (st = check_k(K)) != MMF_OK || (st = check_n(N)) != MMF_OK)
+    return st;
+  if (!aligned(x, 16) || !aligned(Wp, 16) || !aligned(dy, 16) || !aligned(beta, 4) ||
+      (dx && !aligned(dx, 16)) || (dW && !aligned(dW, 16)) || (dnorm_w && !aligned(dnorm_w, 16)) ||
+      (A && !aligned(A, 16)) || (gamma && !aligned(gamma, 4)) || (norm_w && !aligned(norm_w, 16)))
+    return MMF_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < bwd_ws_bytes(T, K, N)) return MMF_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return MMF_ERR_ALIGNMENT;
+  unsigned* status = status_ptr();
+  if (!status) return MMF_ERR_CUDA;
+  BwdCall c;
+  c.x = x;
+  c.xdt = xdt == MMF_F16 ? kInF16 : kInF32;
+  c.T = T;
+  c.K = static_cast<int>(K);
+  c.norm_w = norm_w;
+  c.eps = eps;
+  c.A = A;
+  c.gamma = gamma;
+  c.Wp = Wp;
+  c.beta = beta;
+  c.N = static_cast<int>(N);
+  c.dy = dy;
+  c.dx = dx;
+  c.dxdt = dxdt == MMF_F16 ? kInF16 : kInF32;
+  c.dW = dW;
+  c.dnorm_w = dnorm_w;
+  c.status = status;
+  c.wait_limit_ns = kWaitLimitNs;
+  return from_cuda(launch_bitlinear_backward(c, bwd_ws(ws, T, K, N),
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 MMF_EXPORT mmf_status mmf_ternary_accumulate_i32(const int8_t* A, int64_t T, int64_t K,

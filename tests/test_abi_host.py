@@ -188,3 +188,63 @@ def test_mlgru_quantized_rejects_on_host(kw, code):
         a["I"], a["F"], a["G"], a["xdt"], a["T"], a["H"], a["h0"], a["w"], a["eps"], a["qw"],
         a["qeps"], a["A"], a["gamma"], a["rowsum"], a["hT"], a["ws"], a["wsb"],
         a["stream"]) == code
+
+
+# ------------------------------------------------------------------------------- backward
+def _bwd_base(T, K, N):
+    # codes [T x K], gamma [T], cT [K x N] fp16, dyT [N x T64] fp16, qT [K x T64] fp16,
+    # dxh [T x K] fp32, 1/r [T], norm-weight partials [64 x K], each rounded up to 256 bytes
+    up = lambda v: (v + 255) // 256 * 256
+    t64 = (T + 63) // 64 * 64
+    return (up(T * K) + up(4 * T) + up(2 * K * N) + up(2 * N * t64) + up(2 * K * t64) +
+            up(4 * T * K) + up(4 * T) + up(4 * 64 * K))
+
+
+def test_backward_workspace_sizes():
+    L = mmf.lib()
+    # no split: one partial-free contraction each
+    assert L.mmf_backward_workspace_bytes(17, 256, 384) == _bwd_base(17, 256, 384)
+    assert L.mmf_backward_workspace_bytes(32768, 2048, 2048) == _bwd_base(32768, 2048, 2048)
+    # 2000 tokens, 16 output tiles of dW: its token contraction is split three ways
+    # (3 partial [1024 x 1024] fp32 tiles)
+    assert L.mmf_backward_workspace_bytes(2000, 1024, 1024) == \
+        _bwd_base(2000, 1024, 1024) + 3 * 1024 * 1024 * 4
+    # 300 tokens, 8 output tiles of dxh: its contraction over N = 2048 is split four ways
+    # (4 partial [512 x 1024] tiles, 512 = 300 rounded up to the 256-token tile)
+    assert L.mmf_backward_workspace_bytes(300, 1024, 2048) == \
+        _bwd_base(300, 1024, 2048) + 4 * 512 * 1024 * 4
+    assert L.mmf_backward_workspace_bytes(0, 256, 256) == 0
+    assert L.mmf_backward_workspace_bytes(4, 200, 256) == 0
+    assert L.mmf_backward_workspace_bytes(4, 256, 200) == 0
+
+
+def bwd(**kw):
+    a = dict(x=A16, xdt=1, T=4, K=256, g=None, eps=1e-8, A=None, gamma=None, Wp=A16, beta=A16,
+             N=256, dy=A16, dx=A16, dxdt=0, dW=A16, dg=None, ws=A16, wsb=1 << 24, stream=None)
+    a.update(kw)
+    return mmf.lib().mmf_bitlinear_backward(
+        a["x"], a["xdt"], a["T"], a["K"], a["g"], a["eps"], a["A"], a["gamma"], a["Wp"],
+        a["beta"], a["N"], a["dy"], a["dx"], a["dxdt"], a["dW"], a["dg"], a["ws"], a["wsb"],
+        a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), INVALID), (dict(Wp=None), INVALID), (dict(beta=None), INVALID),
+    (dict(dy=None), INVALID), (dict(dx=None, dW=None, dg=None), INVALID),
+    (dict(A=A16), INVALID), (dict(gamma=A16), INVALID), (dict(xdt=2), INVALID),
+    (dict(dxdt=7), INVALID), (dict(eps=0.0), INVALID), (dict(eps=float("nan")), INVALID),
+    (dict(T=0), SHAPE), (dict(K=192), SHAPE), (dict(N=64), SHAPE), (dict(K=8320), SHAPE),
+    (dict(x=A16 + 8), ALIGN), (dict(dy=A16 + 2), ALIGN), (dict(dx=A16 + 4), ALIGN),
+    (dict(dW=A16 + 8), ALIGN), (dict(dg=A16 + 4), ALIGN), (dict(A=A16 + 1, gamma=A16), ALIGN),
+    (dict(g=A16 + 4), ALIGN), (dict(ws=A16 + 16), ALIGN),
+    (dict(ws=None), WS), (dict(wsb=1000), WS),
+])
+def test_backward_rejects_on_host(kw, code):
+    assert bwd(**kw) == code
+
+
+def test_backward_valid_call_without_gpu_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert bwd() == CUDA
