@@ -302,6 +302,7 @@ prefill_ss_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     const float beta = to_i32 ? 0.0f : (p.beta ? *p.beta : 1.0f);
     const uint32_t accempty0[2] = {map_peer(accempty(0), 0), map_peer(accempty(1), 0)};
     int nbuf = 0;                                      // output tiles used so far (alternating)
+    int last_buf = -1;                                 // tile of the newest committed store
     int n = 0;
     for (int item = tile0; item < n_items; item += tstep, ++n) {
       const int tile = item % p.n_tiles;
@@ -391,7 +392,15 @@ prefill_ss_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         }
         // shared tile: row r = token, 128 bytes, 16-byte chunk k stored at k ^ (r mod 8)
         uint8_t* buf = s_out + (nbuf & 1) * kOutBuf;
-        if (et == 0) bulk_wait_group_read<1>();         // the store that used this tile is read
+        // the newest store that used this tile has read it: one other store may still be
+        // reading the other tile, unless the newest store used this one (stores skipped past
+        // the end break the alternation)
+        if (et == 0) {
+          if (last_buf == (nbuf & 1))
+            bulk_wait_group_read<0>();
+          else
+            bulk_wait_group_read<1>();
+        }
         named_bar_sync(1, 128);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
@@ -402,6 +411,7 @@ prefill_ss_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (et == 0 && tok0 < p.T && col_base + c0 < p.ncols) {
           tma_store_2d(&tm_y, smem_u32(buf), col_base + c0, static_cast<int32_t>(yrow0));
           bulk_commit_group();
+          last_buf = nbuf & 1;
         }
         ++nbuf;
       }
