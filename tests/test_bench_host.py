@@ -33,6 +33,7 @@ def test_profiled_traffic_follows_the_source_hash(tmp_path, monkeypatch):
 def test_committed_summaries_name_a_hash_and_traffic():
     root = os.path.dirname(os.path.abspath(bench.__file__))
     for name in ("program_kernel_hgrn370m_block_t64.md", "program_kernel_hgrn1p3b_decode_t8.md",
-                 "ternary_gemm_hgrn1p3b_prefill_t32768.md", "mlgru_hgrn1p3b_mlgru_t32768.md"):
+                 "ternary_gemm_hgrn1p3b_prefill_t32768.md", "mlgru_hgrn1p3b_mlgru_t32768.md",
+                 "backward_hgrn1p3b_layer_backward_t8192.md"):
         text = open(os.path.join(root, "profiles", name), encoding="utf-8").read()
         assert "source_sha:" in text and "dram_bytes_per_launch:" in text, name
