@@ -708,6 +708,50 @@ def mlgru_bytes(T, H, quantized=False, in_bytes=2):
     return 3 * in_bytes * T * H + out
 
 
+# The MLGRU's gate arithmetic runs on the SM's special-function unit (exp2 and reciprocal):
+# per element three such operations in the chunk-map pass (two exponentials and one
+# reciprocal for both gates) and five in the output pass (the gates again, then the SiLU's
+# exponential and reciprocal).  One call of a single chunk (T <= 32) runs the output pass
+# alone.  The unit issues 16 operations per clock per SM (sm_100, CUDA's arithmetic throughput
+# table); 148 SMs at the 1965 MHz maximum clock give the peak below.
+XU_OPS_PER_CLOCK_PER_SM = 16
+B200_SMS = 148
+B200_MAX_SM_MHZ = 1965.0
+
+
+def xu_peak_ops(sm_mhz=B200_MAX_SM_MHZ):
+    return XU_OPS_PER_CLOCK_PER_SM * B200_SMS * sm_mhz * 1e6
+
+
+def mlgru_xu_ops(T, H):
+    """Special-function-unit operations of one MLGRU call over T tokens of H channels."""
+    per_elem = 5 if T <= 32 else 8
+    return per_elem * T * H
+
+
+def mlgru_roofline(T, H, quantized, ms, hbm_peak, clocks):
+    """Both bounds of one MLGRU call: HBM bytes over the copy peak and special-function-unit
+    operations over that unit's peak.  The binding one (the longer time at peak) is reported
+    as the roofline; the other stays beside it."""
+    nbytes = mlgru_bytes(T, H, quantized)
+    xu = mlgru_xu_ops(T, H)
+    s = ms * 1e-3
+    hbm_ach = nbytes / s / 1e9
+    xu_peak = xu_peak_ops()
+    sm = clocks.get("sm_mhz") if clocks else None
+    hbm = {"bound": "hbm", "achieved": round(hbm_ach, 1), "peak": round(hbm_peak, 1),
+           "unit": "GB/s", "frac": round(hbm_ach / hbm_peak, 4), "bytes_per_call": nbytes,
+           "peak_source": "measured copy bandwidth"}
+    alu = {"bound": "alu", "achieved": round(xu / s / 1e12, 3), "peak": round(xu_peak / 1e12, 3),
+           "unit": "T special-function ops/s", "frac": round(xu / s / xu_peak, 4),
+           "ops_per_call": xu,
+           "peak_source": "16 exp2/reciprocal per clock per SM x 148 SMs x 1965 MHz",
+           "frac_of_clock_scaled_peak": round(xu / s / xu_peak_ops(sm), 4) if sm else None}
+    xu_bound = xu / xu_peak > nbytes / (hbm_peak * 1e9)
+    main, other = (alu, hbm) if xu_bound else (hbm, alu)
+    return dict(main, other_bound=other)
+
+
 def time_mlgru(args, dev, stream, world, local_rank):
     """Times mmf_mlgru_forward and mmf_mlgru_forward_quantized (inputs resident in HBM, larger
     than L2) and one decode token's call."""
@@ -770,18 +814,16 @@ def time_mlgru(args, dev, stream, world, local_rank):
             torch.cuda.synchronize()
             barrier()
         ms = reduce_max(e0.elapsed_time(e1) / n, world, dev)
-        assert mmf.mmf_get_device_status() == 0
-        nbytes = mlgru_bytes(tokens, H, q)
-        achieved = nbytes / (ms * 1e-3) / 1e9
+        if mmf.mmf_get_device_status() != 0:
+            raise RuntimeError("device status reported a timeout in the MLGRU leg")
+        clocks = clk.summary()
+        roof = mlgru_roofline(tokens, H, q, ms, hbm, clocks)
+        roof["kernel"] = "mlgru call (chunk maps, carries, outputs)"
+        roof["traffic"] = profiled_traffic("mlgru", name) if tokens == T else None
         out[label] = {
             "ms_per_call": round(ms, 4), "tokens_per_s": round(tokens * world / (ms * 1e-3), 1),
-            "launches_per_call": 1 if tokens <= 64 else 3, "calls": n,
-            "roofline": {"bound": "hbm", "kernel": "mlgru call (chunk maps, carries, outputs)",
-                         "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
-                         "frac": round(achieved / hbm, 4), "bytes_per_call": nbytes,
-                         "peak_source": "measured copy bandwidth",
-                         "traffic": profiled_traffic("mlgru", name) if tokens == T else None},
-            "clocks": clk.summary()}
+            "launches_per_call": 1 if tokens <= 32 else 3, "calls": n,
+            "roofline": roof, "clocks": clocks}
     del I, F, G, o, A, ws
     torch.cuda.empty_cache()
     return out

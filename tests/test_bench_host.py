@@ -37,3 +37,20 @@ def test_committed_summaries_name_a_hash_and_traffic():
                  "backward_hgrn1p3b_layer_backward_t8192.md"):
         text = open(os.path.join(root, "profiles", name), encoding="utf-8").read()
         assert "source_sha:" in text and "dram_bytes_per_launch:" in text, name
+
+
+def test_mlgru_roofline_takes_the_binding_bound():
+    # 32768 x 2048 fp16 call: 537 MB (82 us at 6546 GB/s) and 8 x 67.1 M special-function
+    # operations (115 us at 16 x 148 x 1965 MHz): the special-function unit binds
+    T, H = 32768, 2048
+    r = bench.mlgru_roofline(T, H, False, 0.259, 6545.9, {"sm_mhz": 1965.0})
+    assert r["bound"] == "alu" and r["other_bound"]["bound"] == "hbm"
+    assert r["ops_per_call"] == 8 * T * H
+    assert abs(r["peak"] - 16 * 148 * 1.965e9 / 1e12) < 1e-3
+    assert abs(r["frac"] - 8 * T * H / 0.259e-3 / (16 * 148 * 1.965e9)) < 1e-4
+    assert abs(r["other_bound"]["frac"] - bench.mlgru_bytes(T, H) / 0.259e-3 / 6545.9e9) < 1e-4
+    # one token: the output pass alone, five operations per element; 16 KB at the copy rate
+    # (2.5 ns) outlasts 10240 operations at the unit's rate (2.2 ns), so HBM is the bound
+    r1 = bench.mlgru_roofline(1, H, False, 0.0066, 6545.9, {})
+    assert r1["bound"] == "hbm" and r1["other_bound"]["ops_per_call"] == 5 * H
+    assert r1["other_bound"]["frac_of_clock_scaled_peak"] is None
