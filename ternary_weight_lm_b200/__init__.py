@@ -6,9 +6,9 @@ PyTorch supplies device memory (``tensor.data_ptr()``) and streams
 is missing, calls raise.
 
 The functions named ``mmf_*`` mirror the C ABI in ``include/mmf.h`` one to one and take
-tensors that the caller owns.  ``quantize_weights``, ``bitlinear_forward`` and
-``bitlinear_glu_forward`` are conveniences that allocate the outputs and the workspace with
-torch and then call the same entry points.
+tensors that the caller owns.  ``quantize_weights``, ``bitlinear_forward``,
+``bitlinear_glu_forward``, ``mlgru_forward`` and ``bitlinear_backward`` are conveniences that
+allocate the outputs and the workspace with torch and then call the same entry points.
 """
 import ctypes
 import os
@@ -24,7 +24,8 @@ __all__ = [
     "mmf_program_workspace_bytes", "mmf_program_init", "mmf_program_run", "Projection",
     "Program", "quantize_weights", "bitlinear_forward", "bitlinear_glu_forward", "workspace",
     "mmf_mlgru_workspace_bytes", "mmf_mlgru_forward", "mmf_mlgru_forward_quantized",
-    "mlgru_forward",
+    "mlgru_forward", "mmf_backward_workspace_bytes", "mmf_bitlinear_backward",
+    "bitlinear_backward",
     "MMF_F32", "MMF_F16", "STATUS",
 ]
 

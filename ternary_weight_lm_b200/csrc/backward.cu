@@ -34,11 +34,19 @@ constexpr int kDgChunks = 64;   // token blocks of the norm-weight gradient's pa
 size_t up256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 int64_t up64(int64_t v) { return (v + 63) / 64 * 64; }
 
+// A 64 x 64 fp16 transpose tile in shared memory, rows of 128 bytes whose 16-byte chunks are
+// permuted by XOR with (row / 8): the column-wise scatter of a transpose (eight rows 8 apart
+// per warp) then falls on eight different bank groups, and every chunk stays 16-byte aligned
+// for the row-wise vector reads.
+__device__ __forceinline__ int tsw(int row, int col) {
+  return row * 64 + ((((col >> 3) ^ (row >> 3)) & 7) << 3) + (col & 7);
+}
+
 // cT[k][n] = c[n][k] as fp16, from the packed codes (layout L1: code 16G + 4i + j of a row at
 // bits 8j + 2i of its 32-bit word G, stored as e = c + 1).  One block per 64 x 64 tile.
 __global__ void __launch_bounds__(256) codes_t_f16_kernel(const uint32_t* __restrict__ wp, int N,
                                                           int K, __half* __restrict__ cT) {
-  __shared__ __align__(16) __half s[64][72];   // [k][n]
+  __shared__ __align__(16) __half s[64 * 64];   // [k][n], swizzled
   const int n0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
   {
     const int rr = threadIdx.x >> 2, ww = threadIdx.x & 3;
@@ -47,7 +55,8 @@ __global__ void __launch_bounds__(256) codes_t_f16_kernel(const uint32_t* __rest
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        s[16 * ww + 4 * i + j][rr] = __int2half_rn(static_cast<int>((w >> (8 * j + 2 * i)) & 3u) - 1);
+        s[tsw(16 * ww + 4 * i + j, rr)] =
+            __int2half_rn(static_cast<int>((w >> (8 * j + 2 * i)) & 3u) - 1);
   }
   __syncthreads();
 #pragma unroll
@@ -55,7 +64,7 @@ __global__ void __launch_bounds__(256) codes_t_f16_kernel(const uint32_t* __rest
     const int idx = threadIdx.x + 256 * h;
     const int row = idx >> 3, ch = idx & 7;
     *reinterpret_cast<uint4*>(cT + static_cast<int64_t>(k0 + row) * N + n0 + ch * 8) =
-        *reinterpret_cast<const uint4*>(&s[row][ch * 8]);
+        *reinterpret_cast<const uint4*>(&s[tsw(row, ch * 8)]);
   }
 }
 
@@ -63,7 +72,7 @@ __global__ void __launch_bounds__(256) codes_t_f16_kernel(const uint32_t* __rest
 __global__ void __launch_bounds__(256) grad_scale_t_kernel(const __half* __restrict__ dy, int64_t T,
                                                            int N, const float* __restrict__ gamma,
                                                            __half* __restrict__ dyT, int64_t ldT) {
-  __shared__ __align__(16) __half s[64][72];   // [n][t]
+  __shared__ __align__(16) __half s[64 * 64];   // [n][t], swizzled
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 64;
   const int n0 = blockIdx.y * 64;
 #pragma unroll
@@ -87,7 +96,7 @@ __global__ void __launch_bounds__(256) grad_scale_t_kernel(const __half* __restr
       for (int e = 0; e < 8; ++e) v[e] = __float2half_rn(0.0f);
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) s[ch * 8 + e][tt] = v[e];
+    for (int e = 0; e < 8; ++e) s[tsw(ch * 8 + e, tt)] = v[e];
   }
   __syncthreads();
 #pragma unroll
@@ -95,14 +104,14 @@ __global__ void __launch_bounds__(256) grad_scale_t_kernel(const __half* __restr
     const int idx = threadIdx.x + 256 * h;
     const int row = idx >> 3, ch = idx & 7;
     *reinterpret_cast<uint4*>(dyT + static_cast<int64_t>(n0 + row) * ldT + t0 + ch * 8) =
-        *reinterpret_cast<const uint4*>(&s[row][ch * 8]);
+        *reinterpret_cast<const uint4*>(&s[tsw(row, ch * 8)]);
   }
 }
 
 // qT[k][t] = q[t][k] as fp16 (exact); columns t >= T of the padded rows are zero.
 __global__ void __launch_bounds__(256) codes_tt_kernel(const int8_t* __restrict__ A, int64_t T,
                                                        int K, __half* __restrict__ qT, int64_t ldT) {
-  __shared__ __align__(16) __half s[64][72];   // [k][t]
+  __shared__ __align__(16) __half s[64 * 64];   // [k][t], swizzled
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 64;
   const int k0 = blockIdx.y * 64;
   {
@@ -112,7 +121,7 @@ __global__ void __launch_bounds__(256) codes_tt_kernel(const int8_t* __restrict_
     if (t < T) raw = __ldcs(reinterpret_cast<const uint4*>(A + t * K + k0 + ch * 16));
     const int8_t* b = reinterpret_cast<const int8_t*>(&raw);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) s[ch * 16 + e][tt] = __int2half_rn(b[e]);
+    for (int e = 0; e < 16; ++e) s[tsw(ch * 16 + e, tt)] = __int2half_rn(b[e]);
   }
   __syncthreads();
 #pragma unroll
@@ -120,7 +129,7 @@ __global__ void __launch_bounds__(256) codes_tt_kernel(const int8_t* __restrict_
     const int idx = threadIdx.x + 256 * h;
     const int row = idx >> 3, ch = idx & 7;
     *reinterpret_cast<uint4*>(qT + static_cast<int64_t>(k0 + row) * ldT + t0 + ch * 8) =
-        *reinterpret_cast<const uint4*>(&s[row][ch * 8]);
+        *reinterpret_cast<const uint4*>(&s[tsw(row, ch * 8)]);
   }
 }
 
