@@ -262,7 +262,7 @@ mmf_status mmf_mlgru_forward_quantized(const void* I, const void* F, const void*
  * to have the call recompute them from x.  dy: fp16 [T x N], row-major.  dx (dxdt f32 or f16),
  * dW and dnorm_w: outputs, each may be NULL to skip it (at least one must be given); they are
  * overwritten, not accumulated into.  ws: mmf_backward_workspace_bytes(T, K, N) bytes, 256-byte
- * aligned.  Errors as for the forward.  Asynchronous on `stream` (up to nine launches). */
+ * aligned.  Errors as for the forward.  Asynchronous on `stream` (up to eleven launches). */
 size_t mmf_backward_workspace_bytes(int64_t T, int64_t K, int64_t N);
 
 mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype xdt, int64_t T, int64_t K,
