@@ -93,9 +93,11 @@ def _check_dg(dg, dg_ref, x, dy, c, beta, eps):
 
 # T from one token to several 256-token tiles with a ragged tail; N and K with an odd number of
 # 128-row halves (the second CTA of a pair reads rows past the end: zeros); K = 7040, the 2.7B
-# down projection's input (27.5 tiles of 256 rows for dxh and dW).
+# down projection's input (27.5 tiles of 256 rows for dxh and dW); the 2.7B gate projection
+# (2560 -> 14080), whose dxh contraction over N is split eight ways.
 @pytest.mark.parametrize("T,K,N", [(1, 128, 128), (17, 256, 384), (300, 1024, 2048),
-                                   (257, 2816, 1024), (130, 7040, 2560), (64, 2048, 5632)])
+                                   (257, 2816, 1024), (130, 7040, 2560), (64, 2048, 5632),
+                                   (33, 2560, 14080)])
 def test_backward_matches_oracle(T, K, N):
     x, g, Wp, beta, c, q, gamma, dy = _problem(T, K, N, seed=T + K + N)
     dx, dW, _ = _gpu(x, g, Wp, beta, q, gamma, dy)
