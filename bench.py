@@ -20,7 +20,10 @@ and, in a "decode" object beside it, the HBM-bound decode workloads (1.3B at 1/8
 2.7B at 8 tokens), each with its own step time, weight GB/s, roofline fraction and clocks.
 An "mlgru" object times the MLGRU recurrence with its swish gate norm (the step after
 i/f/g_proj), alone and fused with o_proj's activation quantisation, on the 1.3B prefill
-shape, and at one decode token.
+shape, and at one decode token; its roofline is the special-function unit, which binds it,
+with HBM beside it.  A "backward" object times the straight-through backward of one 1.3B
+layer's six projections at the prefill length (input- and weight-gradient calls, fp16
+tensor-core contractions) against the measured bf16 dense peak.
 
 Arms:
   default            the CUDA library through its C ABI; the timed region replays CUDA
